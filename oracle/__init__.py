@@ -1,0 +1,213 @@
+"""Orthrus hot-path oracle (fp64, CPU).
+
+TEST INFRASTRUCTURE. Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this package. It shares no code with
+the CUDA path (``diffusion_draft_ar_b200``); the two meet only through the seeded
+input generators in ``diffusion_draft_ar_b200.workloads``.
+
+The arithmetic lives in ``orthrus_oracle.c`` (plain C, fp64, one scalar loop per
+definition); this module compiles it with gcc on first use and marshals numpy
+arrays to it. bf16 tensors travel as their raw 16-bit patterns (``numpy.uint16``).
+
+Definitions followed (Orthrus: Memory-Efficient Parallel Token Generation via
+Dual-View Diffusion, technical summary):
+
+* ``block_attn(view=DIFFUSION)`` -- §2.2, mask M_diff: every block row sees the
+  whole clean prefix and every other block row.
+* ``block_attn(view=VERIFY)`` -- §2.3 item 2: the frozen AR view runs causal
+  attention over the populated block (row i sees block rows 0..i).
+* ``block_attn_split`` -- partial softmax per prefix chunk, merged by the
+  max/sum identity; equal to ``block_attn`` up to rounding.
+* ``consensus`` -- §2.3 item 3: strict left-to-right greedy match, commit up to
+  j-1 plus the AR correction token.
+* ``kv_append`` -- §2.3 item 3 (commit and truncate the cache) and the
+  agents-report.net commentary, "core design" (accepted tokens' KV appended to
+  the shared cache).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+VIEW_DIFFUSION = 0
+VIEW_VERIFY = 1
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "orthrus_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liborthrus_oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile ``orthrus_oracle.c`` into ``liborthrus_oracle.so`` (gcc, -O2, no fast-math)."""
+    stale = (not os.path.exists(_LIB_PATH)) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC)
+    if force or stale:
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-pthread",
+               "-fno-fast-math", "-ffp-contract=off", "-o", tmp, _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def default_threads() -> int:
+    env = os.environ.get("ORTHRUS_ORACLE_THREADS")
+    if env:
+        return max(1, int(env))
+    return max(1, os.cpu_count() or 1)
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        lib = ctypes.CDLL(build())
+        p = ctypes.c_void_p
+        i32, i64, dbl = ctypes.c_int, ctypes.c_int64, ctypes.c_double
+        lib.oracle_block_attn.restype = i32
+        lib.oracle_block_attn.argtypes = [i32] * 8 + [p] * 5 + [p] * 3 + [dbl, i64, p, p, p, i32]
+        lib.oracle_block_attn_split.restype = i32
+        lib.oracle_block_attn_split.argtypes = [i32] * 8 + [p] * 5 + [p] * 3 + [dbl, i64, i64, p, p, p, i32]
+        lib.oracle_consensus.restype = i32
+        lib.oracle_consensus.argtypes = [p, i64, i32, p, p, i32, p, p, p, i32]
+        lib.oracle_kv_append.restype = i32
+        lib.oracle_kv_append.argtypes = [p, p, p, p, p, i32, p, i32, i32, p, p, i32, i32, i32, i32]
+        _lib = lib
+        return lib
+
+
+def _c(a: np.ndarray, dtype) -> np.ndarray:
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def _ptr(a: np.ndarray | None):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _attn_common(view, q_block, k_cache, v_cache, k_block, v_block, prefix_lens, cu_block,
+                 page_table, sel):
+    q = _c(q_block, np.uint16)
+    kc = _c(k_cache, np.uint16)
+    vc = _c(v_cache, np.uint16)
+    kb = _c(k_block, np.uint16)
+    vb = _c(v_block, np.uint16)
+    pl = _c(prefix_lens, np.int32)
+    cu = _c(cu_block, np.int32)
+    pt = _c(page_table, np.int32)
+    if pt.ndim != 2:
+        raise ValueError("page_table must be [B, max_pages_per_seq]")
+    R, Hq, D = q.shape
+    num_pages, Hkv, P, D2 = kc.shape
+    if D2 != D or vc.shape != kc.shape or kb.shape != (R, Hkv, D) or vb.shape != kb.shape:
+        raise ValueError("inconsistent attention shapes")
+    B = pl.shape[0]
+    if cu.shape[0] != B + 1 or int(cu[-1]) != R or pt.shape[0] != B:
+        raise ValueError("inconsistent batch metadata")
+    if sel is None:
+        n_sel, rows, heads = -1, None, None
+        out = np.zeros((R, Hq, D), np.float64)
+    else:
+        rows = _c(sel[0], np.int64)
+        heads = _c(sel[1], np.int32)
+        n_sel = rows.shape[0]
+        out = np.zeros((n_sel, D), np.float64)
+    arrays = (q, kc, vc, kb, vb, pl, cu, pt, rows, heads, out)
+    dims = (int(view), B, Hq, Hkv, D, P, pt.shape[1], num_pages)
+    return dims, arrays, n_sel
+
+
+def block_attn(view, q_block, k_cache, v_cache, k_block, v_block, prefix_lens, cu_block,
+               page_table, scale: float = 0.0, sel=None, threads: int | None = None) -> np.ndarray:
+    """fp64 attention of the block rows over prefix + block keys.
+
+    ``sel`` = (rows int64[n], heads int32[n]) restricts the computation to those
+    (global block row, query head) pairs and returns [n, D]; otherwise [R, Hq, D].
+    """
+    lib = _load()
+    dims, arrs, n_sel = _attn_common(view, q_block, k_cache, v_cache, k_block, v_block,
+                                     prefix_lens, cu_block, page_table, sel)
+    q, kc, vc, kb, vb, pl, cu, pt, rows, heads, out = arrs
+    rc = lib.oracle_block_attn(*dims, _ptr(q), _ptr(kc), _ptr(vc), _ptr(kb), _ptr(vb),
+                               _ptr(pl), _ptr(cu), _ptr(pt), float(scale), n_sel,
+                               _ptr(rows), _ptr(heads), _ptr(out),
+                               threads or default_threads())
+    if rc != 0:
+        raise ValueError(f"oracle_block_attn: bad input (code {rc})")
+    return out
+
+
+def block_attn_split(view, q_block, k_cache, v_cache, k_block, v_block, prefix_lens, cu_block,
+                     page_table, chunk_tokens: int, scale: float = 0.0, sel=None,
+                     threads: int | None = None) -> np.ndarray:
+    """Same as :func:`block_attn`, computed as merged per-chunk partial softmaxes."""
+    lib = _load()
+    dims, arrs, n_sel = _attn_common(view, q_block, k_cache, v_cache, k_block, v_block,
+                                     prefix_lens, cu_block, page_table, sel)
+    q, kc, vc, kb, vb, pl, cu, pt, rows, heads, out = arrs
+    rc = lib.oracle_block_attn_split(*dims, _ptr(q), _ptr(kc), _ptr(vc), _ptr(kb), _ptr(vb),
+                                     _ptr(pl), _ptr(cu), _ptr(pt), float(scale),
+                                     int(chunk_tokens), n_sel, _ptr(rows), _ptr(heads),
+                                     _ptr(out), threads or default_threads())
+    if rc != 0:
+        raise ValueError(f"oracle_block_attn_split: bad input (code {rc})")
+    return out
+
+
+def consensus(logits, draft_tokens, cu_block, threads: int | None = None):
+    """Greedy consensus. Returns (accept_len[B], next_token[B], row_argmax[R]) as int32."""
+    lib = _load()
+    x = np.asarray(logits, dtype=np.float32)
+    if x.ndim != 2:
+        raise ValueError("logits must be [R, ld]")
+    if not x.flags.c_contiguous:
+        x = np.ascontiguousarray(x)
+    R, V = x.shape
+    dr = _c(draft_tokens, np.int32)
+    cu = _c(cu_block, np.int32)
+    B = cu.shape[0] - 1
+    if dr.shape[0] != R or int(cu[-1]) != R:
+        raise ValueError("inconsistent consensus shapes")
+    acc = np.zeros(B, np.int32)
+    nxt = np.zeros(B, np.int32)
+    am = np.zeros(R, np.int32)
+    rc = lib.oracle_consensus(_ptr(x), V, V, _ptr(dr), _ptr(cu), B, _ptr(acc), _ptr(nxt),
+                              _ptr(am), threads or default_threads())
+    if rc != 0:
+        raise ValueError(f"oracle_consensus: bad input (code {rc})")
+    return acc, nxt, am
+
+
+def kv_append(k_block, v_block, cu_block, accept_len, prefix_lens, page_table, k_cache, v_cache,
+              update_lens: bool = True) -> int:
+    """In-place append of the accepted rows into numpy caches (uint16 bf16 bits).
+
+    ``prefix_lens`` (int32 numpy) is updated in place when ``update_lens``.
+    Returns the C status (0 = every index in range).
+    """
+    lib = _load()
+    for name, arr, dt in (("k_cache", k_cache, np.uint16), ("v_cache", v_cache, np.uint16),
+                          ("prefix_lens", prefix_lens, np.int32)):
+        if arr.dtype != dt or not arr.flags.c_contiguous:
+            raise ValueError(f"{name} must be a contiguous {np.dtype(dt).name} array (updated in place)")
+    kb = _c(k_block, np.uint16)
+    vb = _c(v_block, np.uint16)
+    cu = _c(cu_block, np.int32)
+    al = _c(accept_len, np.int32)
+    pt = _c(page_table, np.int32)
+    num_pages, Hkv, P, D = k_cache.shape
+    B = cu.shape[0] - 1
+    return lib.oracle_kv_append(_ptr(kb), _ptr(vb), _ptr(cu), _ptr(al), _ptr(prefix_lens),
+                                int(bool(update_lens)), _ptr(pt), pt.shape[1], num_pages,
+                                _ptr(k_cache), _ptr(v_cache), B, Hkv, D, P)
+
+
+def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
+    """Exact widening of bf16 bit patterns (uint16) to float64."""
+    u = np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16
+    return u.view(np.float32).astype(np.float64)
