@@ -1,0 +1,465 @@
+#!/usr/bin/env python
+"""Throughput of one Orthrus block-decoding round on B200.
+
+A step is one pass of the whole hot path over one batch:
+  block attention (DIFFUSION view) -> block attention (VERIFY view)
+  -> greedy consensus over the verify logits -> KV append of the accepted rows
+on the Qwen3-8B-shaped workload (16 sequences, prefix 8192, block 32, 32/8
+heads, head dim 128, 64-token pages in a random permutation, vocabulary 151936),
+inputs resident in HBM. prefix_lens is restored (64-byte device copy) at the
+start of every step so each step appends at the same positions.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun each rank runs its own batch (weak scaling, no data-path
+collective); rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import datetime
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from diffusion_draft_ar_b200 import workloads as W  # noqa: E402
+
+METRIC = "block-attn KV GB/s (% HBM roofline) at K=32; consensus rows/s; blocks/s"
+UNIT = "GB/s"
+FALLBACK_HBM_GBS = 6650.0
+ATTN_SRC = os.path.join(ROOT, "diffusion_draft_ar_b200", "csrc", "block_attn.cuh")
+TRAFFIC_SUMMARY = os.path.join(ROOT, "profiles", "block_attn_qwen3_8b.md")
+
+
+# ---------------------------------------------------------------------------
+# algorithmic bytes
+
+def attn_bytes(w: W.Workload, m: W.BatchMeta) -> int:
+    """Bytes an ideal kernel moves per call: each prefix K/V element once per
+    (sequence, KV head), plus the block's Q, K, V and the output."""
+    kv = int(m.prefix_lens.to(torch.int64).sum()) * W.cache_bytes_per_token(w)
+    R = m.R
+    return kv + R * w.Hq * w.D * 2 * 2 + R * w.Hkv * w.D * 2 * 2
+
+
+def consensus_bytes(w: W.Workload, m: W.BatchMeta) -> int:
+    return m.R * w.vocab * 4 + m.R * 4 * 2 + m.B * 8
+
+
+def append_bytes(w: W.Workload, accepted: int) -> int:
+    return accepted * w.Hkv * w.D * 2 * 2 * 2  # read + write, K and V
+
+
+def attn_flops(w: W.Workload, m: W.BatchMeta, view: str) -> int:
+    tot = 0
+    for b in range(m.B):
+        L, K = int(m.prefix_lens[b]), int(m.block_lens[b])
+        keys = K * (L + K) if view == "diffusion" else K * L + K * (K + 1) // 2
+        tot += keys * w.Hq
+    return 4 * w.D * tot
+
+
+# ---------------------------------------------------------------------------
+# helpers
+
+def peak_hbm():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            v = float(json.load(f)["hbm_gbs"])
+        return v, "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def traffic_per_launch():
+    """DRAM bytes per attention launch from the committed ncu summary, or None if
+    the summary is missing or was taken on a different kernel source."""
+    try:
+        txt = open(TRAFFIC_SUMMARY).read()
+        src_hash = hashlib.sha256(open(ATTN_SRC, "rb").read()).hexdigest()[:16]
+        m = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]+)", txt)
+        t = re.search(r"dram_bytes_per_launch_full_size:\s*([0-9]+)", txt)
+        if m and t and m.group(1) == src_hash:
+            return int(t.group(1))
+    except Exception:
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, dev_index: int):
+        self.proc = None
+        self.out = None
+        try:
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(dev_index).uuid)
+        except Exception:
+            uuid = None
+        self.cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                    "-lms", "100"] + (["-i", uuid] if uuid else [])
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(self.cmd, stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if not self.proc:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out = ""
+        rows = [l.split(",") for l in out.strip().splitlines() if l.count(",") >= 8]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4)
+                          if r[5 + i].strip().lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle on a bounded sample (reference arm and cpu_baseline)
+
+class OracleSample:
+    """One sequence of the workload: both attention views, its consensus rows and
+    its append, computed by the fp64 CPU oracle."""
+
+    def __init__(self, w: W.Workload, seed: int = 0):
+        import oracle
+        self.oracle = oracle
+        self.w1 = w.with_(B=1)
+        self.wi = W.WorkloadInputs(self.w1, seed=seed)
+        m, r = self.wi.meta, self.wi.rounds[0]
+        self.args = {}
+        for view in W.VIEW_NAMES:
+            self.args[view] = (0 if view == "diffusion" else 1, W.bf16_bits(r.q[view]),
+                               W.bf16_bits(self.wi.k_cache), W.bf16_bits(self.wi.v_cache),
+                               W.bf16_bits(r.k_block[view]), W.bf16_bits(r.v_block[view]),
+                               m.prefix_lens.numpy(), m.cu_block.numpy(), m.page_table.numpy())
+        self.logits = r.logits.numpy()
+        _, _, t = oracle.consensus(self.logits, np.zeros(m.R, np.int32), m.cu_block.numpy())
+        self.drafts = self.wi.drafts(0, torch.from_numpy(t)).numpy()
+        self.kc = W.bf16_bits(self.wi.k_cache).copy()
+        self.vc = W.bf16_bits(self.wi.v_cache).copy()
+        self.bytes = 0
+        for view in W.VIEW_NAMES:
+            self.bytes += attn_bytes(self.w1, m)
+        self.bytes += consensus_bytes(self.w1, m)
+        self.threads = oracle.default_threads()
+
+    def run(self) -> int:
+        o, m = self.oracle, self.wi.meta
+        for view in W.VIEW_NAMES:
+            o.block_attn(*self.args[view], threads=self.threads)
+        acc, _, _ = o.consensus(self.logits, self.drafts, m.cu_block.numpy(), threads=self.threads)
+        lens = m.prefix_lens.numpy().copy()
+        r = self.wi.rounds[0]
+        o.kv_append(W.bf16_bits(r.k_block["verify"]), W.bf16_bits(r.v_block["verify"]),
+                    m.cu_block.numpy(), acc, lens, m.page_table.numpy(), self.kc, self.vc)
+        return self.bytes + append_bytes(self.w1, int(acc.sum()))
+
+
+def cpu_baseline(w: W.Workload, budget_s: float = 10.0) -> dict:
+    s = OracleSample(w)
+    done, nbytes, t0 = 0, 0, time.perf_counter()
+    while True:
+        nbytes += s.run()
+        done += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or done >= w.B:
+            break
+    return {"value": nbytes / el / 1e9, "unit": UNIT, "cores": s.threads, "kind": "oracle",
+            "sample": f"{done} sequence(s) of {w.name} (both attention views over L={w.prefix_len}, "
+                      f"consensus over {w.max_block} rows x V={w.vocab}, append), fp64 C oracle, "
+                      f"{el:.1f} s"}
+
+
+def run_reference(args):
+    world, rank, _ = int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), 0
+    if rank != 0:
+        return
+    w = W.WORKLOADS[args.workload]
+    s = OracleSample(w)
+    for _ in range(args.warmup):
+        s.run()
+    times, nbytes = [], 0
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        nbytes += s.run()
+        times.append(time.perf_counter() - t0)
+    total = sum(times)
+    value = nbytes / total / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": w.name, "sample": "one sequence per step", "B": w.B,
+                   "prefix_len": w.prefix_len, "block": w.block, "Hq": w.Hq, "Hkv": w.Hkv,
+                   "D": w.D, "page_size": w.page_size, "vocab": w.vocab},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": s.threads, "kind": "oracle",
+                         "sample": "one sequence of the workload per step (both views, "
+                                   "consensus, append), fp64 C oracle"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+
+def run_ours(args):
+    world, rank, local = dist_setup()
+    from diffusion_draft_ar_b200 import orthrus as O
+    w = W.WORKLOADS[args.workload]
+    dev = torch.device("cuda", torch.cuda.current_device())
+    wi = W.WorkloadInputs(w, device=dev, seed=rank)
+    m, r = wi.meta, wi.rounds[0]
+    stream = torch.cuda.current_stream()
+    lens0 = m.prefix_lens.to(dev)
+    lens = lens0.clone()
+    cu = m.cu_block.to(dev)
+    table = m.page_table.to(dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    outs, params = {}, {}
+    ws_attn = None
+    for view in W.VIEW_NAMES:
+        outs[view] = torch.empty_like(r.q[view])
+        p = O.attn_params(view, r.q[view], wi.k_cache, wi.v_cache, r.k_block[view],
+                          r.v_block[view], lens, cu, table, outs[view], w.max_block,
+                          kv_split_tokens=w.kv_split_tokens, error_flag=err)
+        n = O.block_attn_workspace_size(p)
+        if ws_attn is None or ws_attn.numel() < n:
+            ws_attn = torch.empty(n, dtype=torch.uint8, device=dev)
+        params[view] = p
+    for p in params.values():
+        p.workspace, p.workspace_bytes = ws_attn.data_ptr(), ws_attn.numel()
+    targets = torch.argmax(r.logits, dim=1).to(torch.int32)
+    drafts = wi.drafts(0, targets)
+    acc = torch.zeros(m.B, dtype=torch.int32, device=dev)
+    nxt = torch.zeros(m.B, dtype=torch.int32, device=dev)
+    ws_cons = torch.empty(O.consensus_workspace_size(m.B, w.max_block, w.vocab),
+                          dtype=torch.uint8, device=dev)
+    L = O.lib
+    sp = ctypes.c_void_p(stream.cuda_stream)
+    P_diff, P_ver = ctypes.byref(params["diffusion"]), ctypes.byref(params["verify"])
+    cons_args = (r.logits.data_ptr(), w.vocab, w.vocab, drafts.data_ptr(), cu.data_ptr(), m.B,
+                 w.max_block, acc.data_ptr(), nxt.data_ptr(), None, ws_cons.data_ptr(),
+                 ws_cons.numel(), sp)
+    kb, vb = r.k_block["verify"], r.v_block["verify"]
+    app_args = (kb.data_ptr(), vb.data_ptr(), cu.data_ptr(), w.max_block, acc.data_ptr(),
+                lens.data_ptr(), 1, table.data_ptr(), m.max_pages, m.num_pages,
+                wi.k_cache.data_ptr(), wi.v_cache.data_ptr(), m.B, w.Hkv, w.D, w.page_size,
+                err.data_ptr(), sp)
+
+    def step(ev=None):
+        lens.copy_(lens0, non_blocking=True)
+        if ev is not None:
+            ev[0].record(stream)
+        s1 = L.orthrus_block_attn(P_diff, sp)
+        if ev is not None:
+            ev[1].record(stream)
+        s2 = L.orthrus_block_attn(P_ver, sp)
+        if ev is not None:
+            ev[2].record(stream)
+        s3 = L.orthrus_consensus(*cons_args)
+        if ev is not None:
+            ev[3].record(stream)
+        s4 = L.orthrus_kv_append(*app_args)
+        if ev is not None:
+            ev[4].record(stream)
+        if s1 or s2 or s3 or s4:
+            raise RuntimeError(f"orthrus call failed: {(s1, s2, s3, s4)} "
+                               f"{L.orthrus_last_error().decode()}")
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if int(err.item()) != 0:
+        raise RuntimeError(f"device error flag {int(err.item())}")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(dev.index)
+    sampler.start()
+    time.sleep(0.3)  # let the sampler take its first reading
+    barrier(world)
+    torch.cuda.synchronize()
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks = sampler.stop()
+    total_ms = t_start.elapsed_time(t_end)
+    part = np.array([[e[j].elapsed_time(e[j + 1]) for j in range(4)] for e in evs])  # ms
+    total_ms = max_over_ranks(total_ms, world)
+    ms_step = total_ms / args.steps
+    t_diff, t_ver, t_cons, t_app = (float(x) for x in part.mean(0))
+
+    accepted = int(acc.sum().item())
+    mean_accept = accepted / m.B
+    b_attn = attn_bytes(w, m)
+    b_step = 2 * b_attn + consensus_bytes(w, m) + append_bytes(w, accepted)
+    value = world * b_step / (ms_step * 1e-3) / 1e9
+    attn_ms = 0.5 * (t_diff + t_ver)
+    attn_gbs = b_attn / (attn_ms * 1e-3) / 1e9
+    peak, peak_src = peak_hbm()
+    flops = 0.5 * (attn_flops(w, m, "diffusion") + attn_flops(w, m, "verify"))
+
+    # ---- end to end through the public API: pinned host inputs in, results out ----
+    e2e_steps = max(1, min(args.steps, args.e2e_steps))
+    h_in = {k: t.cpu().pin_memory() for k, t in (
+        ("qd", r.q["diffusion"]), ("kd", r.k_block["diffusion"]), ("vd", r.v_block["diffusion"]),
+        ("qv", r.q["verify"]), ("kv", r.k_block["verify"]), ("vv", r.v_block["verify"]),
+        ("logits", r.logits), ("drafts", drafts))}
+    d_in = {"qd": r.q["diffusion"], "kd": r.k_block["diffusion"], "vd": r.v_block["diffusion"],
+            "qv": r.q["verify"], "kv": r.k_block["verify"], "vv": r.v_block["verify"],
+            "logits": r.logits, "drafts": drafts}
+    h_out = {"od": torch.empty_like(outs["diffusion"], device="cpu").pin_memory(),
+             "ov": torch.empty_like(outs["verify"], device="cpu").pin_memory(),
+             "acc": torch.empty_like(acc, device="cpu").pin_memory(),
+             "nxt": torch.empty_like(nxt, device="cpu").pin_memory()}
+    d_out = {"od": outs["diffusion"], "ov": outs["verify"], "acc": acc, "nxt": nxt}
+    h2d = sum(t.numel() * t.element_size() for t in h_in.values())
+    d2h = sum(t.numel() * t.element_size() for t in h_out.values())
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        for k in h_in:
+            d_in[k].copy_(h_in[k], non_blocking=True)
+        step()
+        for k in h_out:
+            h_out[k].copy_(d_out[k], non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / e2e_steps
+    e2e_value = world * b_step / (e2e_ms * 1e-3) / 1e9
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, budget_s=args.cpu_seconds)
+
+    if rank == 0:
+        roof = {"bound": "hbm", "achieved": attn_gbs, "peak": peak, "unit": "GB/s",
+                "frac": attn_gbs / peak, "traffic": traffic_per_launch(),
+                "kernel": "orthrus_block_attn (attention + split combine), mean of both views",
+                "algorithmic_bytes_per_launch": b_attn, "us_per_launch": attn_ms * 1e3,
+                "peak_source": f"{peak_src} HBM copy bandwidth",
+                "tensor_tflops": flops / (attn_ms * 1e-3) / 1e12}
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) bf16 Q/K/V, fp32 logits; no weights)",
+            "config": {"workload": w.name, "B": w.B, "prefix_len": w.prefix_len, "block": w.block,
+                       "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D, "page_size": w.page_size,
+                       "vocab": w.vocab, "pages": "random permutation",
+                       "parallelism": f"dp{world} (independent batches)",
+                       "l2": "inputs larger than L2 (KV cache 537 MB, logits 311 MB), no flush"},
+            "block_attn_gbs": attn_gbs, "block_attn_us": {"diffusion": t_diff * 1e3,
+                                                          "verify": t_ver * 1e3},
+            "consensus_rows_per_s": world * m.R / (t_cons * 1e-3),
+            "consensus_us": t_cons * 1e3, "kv_append_us": t_app * 1e3,
+            "blocks_per_s": world * m.B / (ms_step * 1e-3),
+            "tokens_verified_per_s": world * m.R / (t_ver * 1e-3),
+            "mean_accept_len": mean_accept,
+            "roofline": roof,
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "steps": e2e_steps, "ms_per_step": e2e_ms,
+                    "note": "per step: pinned H2D of both views' q/k/v blocks, logits and drafts; "
+                            "D2H of both outputs, accept lengths and next tokens; "
+                            "the KV cache stays resident"},
+            "gpu_launches": args.steps * 7,
+            "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="qwen3_8b", choices=sorted(W.WORKLOADS))
+    ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,840 @@
+// Orthrus block attention on sm_100a: tcgen05 MMAs with TMEM accumulators,
+// TMA-fed shared-memory pipeline, warp-specialised roles, split-KV partials.
+//
+// What it computes ("Orthrus: Memory-Efficient Parallel Token Generation via
+// Dual-View Diffusion", technical summary §2.2 mask M_diff for the DIFFUSION
+// view and §2.3 item 2 for the VERIFY view): for every sequence b, KV head h,
+// block row i and query head h*G+g, softmax attention over the L_b prefix keys
+// read through the page table followed by the block's own K_b keys, the block
+// keys being all visible (DIFFUSION) or visible up to row i (VERIFY).
+//
+// Work unit = (sequence b, KV head h). Its G*K_b query rows (token-major:
+// row r = i*G + g) form one M = 128 MMA tile that stays in shared memory; the
+// unit's keys are cut into 64-key tiles: ceil(L_b/64) prefix tiles, then one
+// block tile. A CTA (one per SM) walks a contiguous range of the global
+// (unit, tile) sequence, so every CTA gets the same number of tiles whatever
+// the prefix lengths; a unit cut by a range boundary is finished by the combine
+// kernel from per-CTA partials (max, sum, normalised accumulator).
+//
+// Roles (320 threads):
+//   warp 0      TMA producer: Q tile per unit, K and V tiles into a ring of
+//               stages, page ids read from the page table.
+//   warp 1      MMA issuer: S = Q K^T into TMEM, then O += P V; owns TMEM.
+//   warps 2-5   softmax group 0 (even tiles), warps 6-9 softmax group 1 (odd
+//               tiles). Each thread owns one query row (= one TMEM lane): it
+//               reads its S row from TMEM, applies the view's mask, keeps a
+//               running max/sum, writes P (bf16) to shared memory for the PV
+//               MMA and, at the end of a unit, merges the two groups'
+//               accumulators and stores the output (or a partial).
+// The two softmax groups keep separate O accumulators (TMEM columns), so they
+// never wait on each other inside a unit.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "orthrus.h"
+#include "ptx.cuh"
+
+namespace orthrus {
+
+constexpr int kTileN = 64;          // keys per tile
+constexpr int kTileM = 128;         // query rows per MMA tile
+constexpr int kAttnThreads = 320;   // 10 warps
+constexpr int kProducerWarp = 0;
+constexpr int kMmaWarp = 1;
+constexpr int kSoftmaxWarp0 = 2;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTmemS = 0;      // S of group w at column 64*w
+constexpr uint32_t kTmemO = 128;    // O of group w at column 128 + D*w
+constexpr uint32_t kTmemX = 384;    // (max, sum) exchange between groups
+constexpr float kRescaleLog2 = 8.0f;  // rescale O only when the max grows by > 2^8
+
+struct AttnArgs {
+  int view, B, Hq, Hkv, G, page_size, max_pages, num_pages, max_block, total_rows;
+  const int* prefix_lens;
+  const int* cu_block;
+  const int* page_table;
+  __nv_bfloat16* out;
+  float* ws_o;     // partial accumulators [parts][128][D]
+  float* ws_lse;   // partial log2-sum-exp  [parts][128]
+  int* error_flag;
+  float scale_log2;  // softmax scale * log2(e)
+  int q_box_rows;    // tokens per Q box: min(max_block, total_rows)
+  int blk_box_rows;  // rows per block-K/V box: min(64, total_rows)
+  int chunked;       // 0: balanced ranges over num_ctas CTAs; 1: fixed chunks
+  int chunk_tiles;   // chunked: prefix tiles per chunk
+  int max_chunks;    // chunked: chunks per unit (grid = B * Hkv * max_chunks)
+  int num_ctas;      // grid size
+  unsigned long long timeout_ns;
+};
+
+// ---------------------------------------------------------------------------
+// Schedule: identical arithmetic in every role and in the combine kernel.
+
+// K_b; 0 for a sequence whose row range is malformed (it is skipped and flagged).
+__device__ __forceinline__ int seq_block_len(const AttnArgs& a, int b) {
+  if (!a.cu_block) return a.max_block;
+  const int r0 = a.cu_block[b], r1 = a.cu_block[b + 1];
+  if (r0 < 0 || r1 < r0 || r1 > a.total_rows || r1 - r0 > a.max_block) return 0;
+  return r1 - r0;
+}
+__device__ __forceinline__ bool seq_rows_bad(const AttnArgs& a, int b) {
+  if (!a.cu_block) return false;
+  const int r0 = a.cu_block[b], r1 = a.cu_block[b + 1];
+  return r0 < 0 || r1 < r0 || r1 > a.total_rows || r1 - r0 > a.max_block;
+}
+__device__ __forceinline__ int seq_row0(const AttnArgs& a, int b) {
+  return a.cu_block ? a.cu_block[b] : b * a.max_block;
+}
+// Prefix length clamped to what the page table can address.
+__device__ __forceinline__ int seq_prefix_len(const AttnArgs& a, int b) {
+  const int L = a.prefix_lens[b];
+  const long long cap = (long long)a.max_pages * a.page_size;
+  return L < 0 ? 0 : (L > cap ? (int)cap : L);
+}
+__device__ __forceinline__ bool seq_len_bad(const AttnArgs& a, int b) {
+  const int L = a.prefix_lens[b];
+  return L < 0 || (long long)L > (long long)a.max_pages * a.page_size;
+}
+__device__ __forceinline__ int seq_tiles(const AttnArgs& a, int b) {
+  if (seq_block_len(a, b) <= 0) return 0;
+  return (seq_prefix_len(a, b) + kTileN - 1) / kTileN + 1;
+}
+// Chunked mode: number of chunks of a unit with nt tiles (block tile joins the last).
+__device__ __forceinline__ int unit_chunks(const AttnArgs& a, int nt) {
+  const int np = nt - 1;
+  const int c = (np + a.chunk_tiles - 1) / a.chunk_tiles;
+  return c < 1 ? 1 : c;
+}
+
+__device__ __forceinline__ long long total_tiles(const AttnArgs& a) {
+  long long T = 0;
+  for (int b = 0; b < a.B; ++b) T += (long long)a.Hkv * seq_tiles(a, b);
+  return T;
+}
+__device__ __forceinline__ long long range_begin(long long T, int c, int C) {
+  return T * c / C;
+}
+
+struct Segment {
+  int b, h, t0, t1, nt;
+  int part;  // -1: the CTA covers the whole unit and writes the output
+};
+
+struct SegCursor {
+  int b, h, t;
+  long long remaining;
+  int first;
+  int cta;
+};
+
+__device__ __forceinline__ void cursor_init(const AttnArgs& a, int cta, SegCursor& c) {
+  c.cta = cta;
+  c.first = 1;
+  c.b = a.B;
+  c.h = 0;
+  c.t = 0;
+  c.remaining = 0;
+  if (a.chunked) {
+    const int chunk = cta % a.max_chunks;
+    const int u = cta / a.max_chunks;
+    const int b = u / a.Hkv;
+    if (b >= a.B) return;
+    const int nt = seq_tiles(a, b);
+    if (nt == 0 || chunk >= unit_chunks(a, nt)) return;
+    c.b = b;
+    c.h = u % a.Hkv;
+    c.t = chunk * a.chunk_tiles;
+    c.remaining = (chunk == unit_chunks(a, nt) - 1) ? (nt - c.t) : a.chunk_tiles;
+    return;
+  }
+  const long long T = total_tiles(a);
+  const long long g0 = range_begin(T, cta, a.num_ctas);
+  c.remaining = range_begin(T, cta + 1, a.num_ctas) - g0;
+  if (c.remaining <= 0) return;
+  long long acc = 0;
+  for (int b = 0; b < a.B; ++b) {
+    const int nt = seq_tiles(a, b);
+    const long long U = (long long)a.Hkv * nt;
+    if (g0 < acc + U) {
+      const long long off = g0 - acc;
+      c.b = b;
+      c.h = (int)(off / nt);
+      c.t = (int)(off % nt);
+      return;
+    }
+    acc += U;
+  }
+  c.remaining = 0;
+}
+
+__device__ __forceinline__ bool cursor_next(const AttnArgs& a, SegCursor& c, Segment& s) {
+  if (c.remaining <= 0 || c.b >= a.B) return false;
+  const int nt = seq_tiles(a, c.b);
+  long long end = c.t + c.remaining;
+  const int t1 = end < nt ? (int)end : nt;
+  s.b = c.b;
+  s.h = c.h;
+  s.t0 = c.t;
+  s.t1 = t1;
+  s.nt = nt;
+  const bool full = (s.t0 == 0 && s.t1 == nt);
+  s.part = full ? -1 : (a.chunked ? c.cta : c.cta * 2 + (c.first ? 0 : 1));
+  c.first = 0;
+  c.remaining -= (t1 - c.t);
+  c.t = 0;
+  if (++c.h == a.Hkv) {
+    c.h = 0;
+    do {
+      ++c.b;
+    } while (c.b < a.B && seq_tiles(a, c.b) == 0);
+  }
+  return true;
+}
+
+// ---------------------------------------------------------------------------
+// Shared-memory layout (offsets from a 1024-byte aligned base).
+
+template <int D>
+struct AttnLayout {
+  static constexpr int DH = D / 64;                   // 64-column panels per row
+  static constexpr int kStages = (D == 128) ? 5 : 8;  // K/V ring depth
+  static constexpr int kQPanel = kTileM * 128;        // bytes of one Q panel
+  static constexpr int kQBytes = DH * kQPanel;
+  static constexpr int kPBytes = kTileM * kTileN * 2;  // one group's P tile
+  static constexpr int kKVPanel = kTileN * 128;        // bytes of one K (or V) panel
+  static constexpr int kKVBytes = DH * kKVPanel;       // one K (or V) tile
+  static constexpr int kQOff = 0;
+  static constexpr int kPOff = kQOff + kQBytes;
+  static constexpr int kKOff = kPOff + 2 * kPBytes;
+  static constexpr int kVOff = kKOff + kStages * kKVBytes;
+  static constexpr int kBarOff = kVOff + kStages * kKVBytes;
+  // barrier indices
+  static constexpr int kBarKvFull = 0;
+  static constexpr int kBarKvEmpty = kStages;
+  static constexpr int kBarQFull = 2 * kStages;
+  static constexpr int kBarQEmpty = kBarQFull + 1;
+  static constexpr int kBarSFull = kBarQEmpty + 1;    // [2]
+  static constexpr int kBarPReady = kBarSFull + 2;    // [2]
+  static constexpr int kBarOReady = kBarPReady + 2;   // [2]
+  static constexpr int kBarOFree = kBarOReady + 2;
+  static constexpr int kBarXchg = kBarOFree + 1;
+  static constexpr int kBarDrain = kBarXchg + 1;
+  static constexpr int kNumBars = kBarDrain + 1;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;  // abort flag, TMEM base
+  static constexpr int kBytes = kMiscOff + 16;
+  static constexpr int kAlloc = kBytes + 1024;  // slack to align the base
+  static_assert(kAlloc <= 232448, "shared memory budget exceeded");
+};
+
+// Descriptors of the four MMA operands (all SWIZZLE_128B).
+// A = Q (K-major): panel p at +p*kQPanel, 8-row groups 1024 B apart.
+// B = K tile (K-major): panel p at +p*kKVPanel.
+// A = P (K-major): one 64-key panel.
+// B = V tile (MN-major): D-panels kKVPanel apart (LBO), 8-key groups 1024 B apart (SBO).
+template <int D>
+__device__ __forceinline__ uint64_t desc_q(uint32_t q, int kk) {
+  return smem_desc_sw128(q + (kk >> 2) * AttnLayout<D>::kQPanel + (kk & 3) * 32, 16, 1024);
+}
+template <int D>
+__device__ __forceinline__ uint64_t desc_k(uint32_t k, int kk) {
+  return smem_desc_sw128(k + (kk >> 2) * AttnLayout<D>::kKVPanel + (kk & 3) * 32, 16, 1024);
+}
+__device__ __forceinline__ uint64_t desc_p(uint32_t p, int kk) {
+  return smem_desc_sw128(p + kk * 32, 16, 1024);
+}
+template <int D>
+__device__ __forceinline__ uint64_t desc_v(uint32_t v, int kk) {
+  return smem_desc_sw128(v + kk * 16 * 128, AttnLayout<D>::kKVPanel, 1024);
+}
+
+// Keys of tile t that exist: 64 for a full prefix tile, fewer for the last
+// partial prefix tile, K_b for the block tile.
+__device__ __forceinline__ int tile_valid_keys(int t, int L, int np, int Kb) {
+  if (t == np) return Kb;
+  const int rem = L - t * kTileN;
+  return rem < kTileN ? rem : kTileN;
+}
+
+__device__ __forceinline__ void raise_flag(const AttnArgs& a, int bits) {
+  if (a.error_flag) atomicOr(a.error_flag, bits);
+}
+
+// ---------------------------------------------------------------------------
+// Roles
+
+template <int D>
+__device__ __forceinline__ void producer_role(const AttnArgs& a, uint8_t* smem,
+                                              const CUtensorMap* tm_q, const CUtensorMap* tm_kc,
+                                              const CUtensorMap* tm_vc, const CUtensorMap* tm_kb,
+                                              const CUtensorMap* tm_vb, volatile int* abort_flag) {
+  using Lay = AttnLayout<D>;
+  const uint32_t base = smem_u32(smem);
+  const uint32_t bars = base + Lay::kBarOff;
+  auto bar = [&](int i) { return bars + 8u * i; };
+  int issued[Lay::kStages];
+#pragma unroll
+  for (int s = 0; s < Lay::kStages; ++s) issued[s] = 0;
+  int q_issued = 0;
+  bool ok = true;
+
+  SegCursor cur;
+  cursor_init(a, blockIdx.x, cur);
+  Segment sg;
+  int it = 0, si = 0;
+  while (ok && cursor_next(a, cur, sg)) {
+    const int b = sg.b, h = sg.h;
+    const int Kb = seq_block_len(a, b), row0 = seq_row0(a, b);
+    const int L = seq_prefix_len(a, b);
+    const int np = (L + kTileN - 1) / kTileN;
+    (void)Kb;
+    // Q tile of this unit: rows (i, g) for i < max_block, g < G.
+    if (si > 0 && !mbar_wait(bar(Lay::kBarQEmpty), (si - 1) & 1, abort_flag, a.timeout_ns)) {
+      ok = false;
+      break;
+    }
+    mbar_arrive_expect_tx(bar(Lay::kBarQFull), Lay::DH * a.G * a.q_box_rows * 128);
+    for (int p = 0; p < Lay::DH; ++p)
+      tma_load_3d(base + Lay::kQOff + p * Lay::kQPanel, tm_q, bar(Lay::kBarQFull), p * 64,
+                  h * a.G, row0);
+    ++q_issued;
+    for (int t = sg.t0; t < sg.t1; ++t, ++it) {
+      const int stage = it % Lay::kStages;
+      const int round = it / Lay::kStages;
+      if (round > 0 &&
+          !mbar_wait(bar(Lay::kBarKvEmpty + stage), (round - 1) & 1, abort_flag, a.timeout_ns)) {
+        ok = false;
+        break;
+      }
+      const uint32_t fb = bar(Lay::kBarKvFull + stage);
+      const uint32_t kdst = base + Lay::kKOff + stage * Lay::kKVBytes;
+      const uint32_t vdst = base + Lay::kVOff + stage * Lay::kKVBytes;
+      mbar_arrive_expect_tx(fb, t < np ? 2 * Lay::kKVBytes : 2 * Lay::DH * a.blk_box_rows * 128);
+      ++issued[stage];
+      if (t < np) {
+        const int tok = t * kTileN;
+        const int pidx = tok / a.page_size;
+        int page = a.page_table[(long long)b * a.max_pages + pidx];
+        if (page < 0 || page >= a.num_pages) {
+          raise_flag(a, ORTHRUS_FLAG_BAD_PAGE);
+          page = 0;  // keep the pipeline flowing on an in-bounds page
+        }
+        const int row = (page * a.Hkv + h) * a.page_size + (tok % a.page_size);
+        for (int p = 0; p < Lay::DH; ++p) {
+          tma_load_2d(kdst + p * Lay::kKVPanel, tm_kc, fb, p * 64, row);
+          tma_load_2d(vdst + p * Lay::kKVPanel, tm_vc, fb, p * 64, row);
+        }
+      } else {
+        for (int p = 0; p < Lay::DH; ++p) {
+          tma_load_3d(kdst + p * Lay::kKVPanel, tm_kb, fb, p * 64, h, row0);
+          tma_load_3d(vdst + p * Lay::kKVPanel, tm_vb, fb, p * 64, h, row0);
+        }
+      }
+    }
+    ++si;
+  }
+  if (!ok || *abort_flag) {
+    // Wind down: let every copy this thread started land before the CTA exits.
+    volatile int no_abort = 0;
+    for (int s = 0; s < Lay::kStages; ++s)
+      if (issued[s] > 0)
+        mbar_wait(bar(Lay::kBarKvFull + s), (issued[s] - 1) & 1, &no_abort, 20000000ull);
+    if (q_issued > 0) mbar_wait(bar(Lay::kBarQFull), (q_issued - 1) & 1, &no_abort, 20000000ull);
+  }
+}
+
+// One step of the MMA issuer's walk over the CTA's tiles.
+struct TileStep {
+  SegCursor cur;
+  Segment sg;
+  int si, t, it, L, np, Kb;
+  bool valid;
+};
+
+__device__ __forceinline__ bool step_next(const AttnArgs& a, TileStep& s) {
+  if (s.valid && s.t + 1 < s.sg.t1) {
+    ++s.t;
+    ++s.it;
+    return true;
+  }
+  if (!cursor_next(a, s.cur, s.sg)) {
+    s.valid = false;
+    return false;
+  }
+  ++s.si;
+  ++s.it;
+  s.t = s.sg.t0;
+  s.L = seq_prefix_len(a, s.sg.b);
+  s.np = (s.L + kTileN - 1) / kTileN;
+  s.Kb = seq_block_len(a, s.sg.b);
+  s.valid = true;
+  return true;
+}
+
+template <int D>
+__device__ __forceinline__ void mma_role(const AttnArgs& a, uint8_t* smem, uint32_t tmem,
+                                         volatile int* abort_flag) {
+  using Lay = AttnLayout<D>;
+  const int lane = threadIdx.x & 31;
+  const uint32_t base = smem_u32(smem);
+  const uint32_t bars = base + Lay::kBarOff;
+  auto bar = [&](int i) { return bars + 8u * i; };
+  constexpr uint32_t kIdescQK = idesc_bf16_f32(kTileM, kTileN, 0);
+  constexpr uint32_t kIdescPV = idesc_bf16_f32(kTileM, D, 1);
+
+  // Lane 0 waits; the verdict is shared so the warp stays converged.
+  auto wait = [&](uint32_t b, uint32_t parity) -> bool {
+    int ok = 1;
+    if (lane == 0) ok = mbar_wait(b, parity, abort_flag, a.timeout_ns) ? 1 : 0;
+    return __shfl_sync(0xffffffffu, ok, 0) != 0;
+  };
+
+  auto issue_qk = [&](const TileStep& j) -> bool {
+    const int stage = j.it % Lay::kStages;
+    if (j.t == j.sg.t0 && !wait(bar(Lay::kBarQFull), j.si & 1)) return false;
+    if (!wait(bar(Lay::kBarKvFull + stage), (j.it / Lay::kStages) & 1)) return false;
+    tc_fence_after();
+    if (lane == 0) {
+      const uint32_t q = base + Lay::kQOff;
+      const uint32_t k = base + Lay::kKOff + stage * Lay::kKVBytes;
+      const uint32_t d = tmem + kTmemS + 64u * (j.it & 1);
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk)
+        mma_bf16_ss(d, desc_q<D>(q, kk), desc_k<D>(k, kk), kIdescQK, kk > 0 ? 1u : 0u);
+      mma_commit(bar(Lay::kBarSFull + (j.it & 1)));
+      if (j.t == j.sg.t1 - 1) mma_commit(bar(Lay::kBarQEmpty));
+    }
+    __syncwarp();
+    return true;
+  };
+
+  auto issue_pv = [&](const TileStep& j) -> bool {
+    const int w = j.it & 1;
+    const int stage = j.it % Lay::kStages;
+    if (!wait(bar(Lay::kBarPReady + w), (j.it >> 1) & 1)) return false;
+    if (j.t == j.sg.t0 && j.si > 0 && !wait(bar(Lay::kBarOFree), (j.si - 1) & 1)) return false;
+    const int nvalid = tile_valid_keys(j.t, j.L, j.np, j.Kb);
+    const uint32_t v = base + Lay::kVOff + stage * Lay::kKVBytes;
+    if (nvalid < kTileN) {
+      // Rows past the last valid key may hold stale or non-finite data;
+      // P is zero there, but 0 * NaN is NaN, so clear those V rows.
+      const int rows = kTileN - nvalid;
+      const int chunks = rows * Lay::DH * 8;  // 16-byte chunks
+      for (int c = lane; c < chunks; c += 32) {
+        const int p = c / (rows * 8);
+        const int rem = c % (rows * 8);
+        const int r = nvalid + rem / 8;
+        st_shared_v4(v + p * Lay::kKVPanel + r * 128 + (rem % 8) * 16, 0u, 0u, 0u, 0u);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+    }
+    tc_fence_after();
+    if (lane == 0) {
+      const uint32_t pbuf = base + Lay::kPOff + w * Lay::kPBytes;
+      const uint32_t d = tmem + kTmemO + (uint32_t)(D * w);
+      const uint32_t acc0 = (j.t - j.sg.t0 >= 2) ? 1u : 0u;
+#pragma unroll
+      for (int kk = 0; kk < kTileN / 16; ++kk)
+        mma_bf16_ss(d, desc_p(pbuf, kk), desc_v<D>(v, kk), kIdescPV, (kk > 0) ? 1u : acc0);
+      mma_commit(bar(Lay::kBarOReady + w));
+      mma_commit(bar(Lay::kBarKvEmpty + stage));
+    }
+    __syncwarp();
+    return true;
+  };
+
+  TileStep qs, ps;
+  cursor_init(a, blockIdx.x, qs.cur);
+  qs.si = -1;
+  qs.it = -1;
+  qs.valid = false;
+  ps = qs;
+  bool ok = true;
+  if (step_next(a, qs)) ok = issue_qk(qs);
+  while (ok && step_next(a, ps)) {
+    const bool have_next = step_next(a, qs);
+    const bool same_seg = have_next && qs.si == ps.si;
+    if (same_seg) ok = issue_qk(qs);
+    if (ok) ok = issue_pv(ps);
+    if (ok && have_next && !same_seg) ok = issue_qk(qs);
+  }
+  // Drain: every MMA issued above completes before TMEM is released.
+  if (lane == 0) {
+    mma_commit(bar(Lay::kBarDrain));
+    volatile int no_abort = 0;
+    mbar_wait(bar(Lay::kBarDrain), 0, &no_abort, 20000000ull);
+  }
+  __syncwarp();
+}
+
+template <int D>
+__device__ __forceinline__ void softmax_role(const AttnArgs& a, uint8_t* smem, uint32_t tmem,
+                                             volatile int* abort_flag) {
+  using Lay = AttnLayout<D>;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int w = (warp - kSoftmaxWarp0) >> 2;   // softmax group 0 or 1
+  const int row = 32 * (warp & 3) + lane;      // query row == TMEM lane
+  const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
+  const uint32_t base = smem_u32(smem);
+  const uint32_t bars = base + Lay::kBarOff;
+  auto bar = [&](int i) { return bars + 8u * i; };
+  const uint32_t t_s = tmem + lane_off + kTmemS + 64u * w;
+  const uint32_t t_o_self = tmem + lane_off + kTmemO + (uint32_t)(D * w);
+  const uint32_t t_o0 = tmem + lane_off + kTmemO;
+  const uint32_t t_o1 = tmem + lane_off + kTmemO + D;
+  const uint32_t pbuf = base + Lay::kPOff + w * Lay::kPBytes;
+  const float c = a.scale_log2;
+  const float NEG_INF = -__int_as_float(0x7f800000);
+
+  auto wait = [&](uint32_t b, uint32_t parity) -> bool {
+    const bool ok = mbar_wait(b, parity, abort_flag, a.timeout_ns);
+    return __all_sync(0xffffffffu, ok);
+  };
+
+  int cnt = 0;        // tiles this group processed (CTA-wide)
+  int pv_waited = 0;  // PV completions of this group already observed
+
+  SegCursor cur;
+  cursor_init(a, blockIdx.x, cur);
+  Segment sg;
+  int it = 0, si = 0;
+  bool ok = true;
+  while (ok && cursor_next(a, cur, sg)) {
+    const int b = sg.b, h = sg.h;
+    const int Kb = seq_block_len(a, b), row0 = seq_row0(a, b);
+    const int L = seq_prefix_len(a, b);
+    const int np = (L + kTileN - 1) / kTileN;
+    const int rows_valid = a.G * Kb;
+    const bool my_valid = row < rows_valid;
+    const int irow = row / a.G;   // block row (token) of this query row
+    const int ntile = sg.t1 - sg.t0;
+    const bool has0 = ntile >= 2 || ((it & 1) == 0);
+    const bool has1 = ntile >= 2 || ((it & 1) == 1);
+    float m_ref = NEG_INF, l_sum = 0.f;
+    bool has = false;
+
+    for (int t = sg.t0; t < sg.t1; ++t, ++it) {
+      if ((it & 1) != w) continue;
+      if (!wait(bar(Lay::kBarSFull + w), (it >> 1) & 1)) { ok = false; break; }
+      tc_fence_after();
+      float s[64];
+      tmem_ld32(t_s, *reinterpret_cast<float(*)[32]>(&s[0]));
+      tmem_ld32(t_s + 32, *reinterpret_cast<float(*)[32]>(&s[32]));
+      tmem_wait_ld();
+      // mask: keys that do not exist or that this row may not see
+      int lim = kTileN;
+      if (!my_valid) lim = 0;
+      else if (t == np) lim = (a.view == ORTHRUS_VIEW_DIFFUSION) ? Kb : (irow + 1);
+      else if (t == np - 1) lim = L - t * kTileN;
+      if (lim < kTileN) {
+#pragma unroll
+        for (int k = 0; k < 64; ++k) s[k] = (k < lim) ? s[k] : NEG_INF;
+      }
+      float mt = NEG_INF;
+#pragma unroll
+      for (int k = 0; k < 64; ++k) mt = fmaxf(mt, s[k]);
+      const float m_new = fmaxf(m_ref, mt * c);
+      const bool need = has && (m_new > m_ref + kRescaleLog2);
+      if (!has) m_ref = m_new;
+      // The previous PV of this group must be done before P is overwritten
+      // (and before O is rescaled).
+      if (cnt > 0 && pv_waited < cnt) {
+        if (!wait(bar(Lay::kBarOReady + w), pv_waited & 1)) { ok = false; break; }
+        ++pv_waited;
+      }
+      if (__any_sync(0xffffffffu, need)) {
+        const float alpha = need ? ex2_approx(m_ref - m_new) : 1.f;
+        if (need) {
+          l_sum *= alpha;
+          m_ref = m_new;
+        }
+        tc_fence_after();
+#pragma unroll 1
+        for (int ch = 0; ch < D / 32; ++ch) {
+          float o[32];
+          tmem_ld32(t_o_self + 32 * ch, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int k = 0; k < 32; ++k) o[k] *= alpha;
+          tmem_st32(t_o_self + 32 * ch, o);
+        }
+        tmem_wait_st();
+      }
+      const float mref = (m_ref == NEG_INF) ? 0.f : m_ref;
+      float rsum = 0.f;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        float p[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          p[k] = ex2_approx(fmaf(s[8 * q + k], c, -mref));
+          rsum += p[k];
+        }
+        const uint32_t addr = pbuf + row * 128 + ((q ^ (row & 7)) << 4);
+        st_shared_v4(addr, pack_bf16x2(p[0], p[1]), pack_bf16x2(p[2], p[3]),
+                     pack_bf16x2(p[4], p[5]), pack_bf16x2(p[6], p[7]));
+      }
+      l_sum += rsum;
+      has = true;
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(bar(Lay::kBarPReady + w));
+      ++cnt;
+    }
+    if (!ok) break;
+
+    // ---- end of the unit: merge the two groups, store output or partial ----
+    if (pv_waited < cnt) {
+      if (!wait(bar(Lay::kBarOReady + w), pv_waited & 1)) { ok = false; break; }
+      ++pv_waited;
+    }
+    {
+      float x[32];
+      x[0] = m_ref;
+      x[1] = l_sum;
+      // only columns 0..1 matter; a 32-column store keeps one code path
+#pragma unroll
+      for (int k = 2; k < 32; ++k) x[k] = 0.f;
+      tmem_st32(tmem + lane_off + kTmemX + 32u * ((si & 1) * 2 + w), x);
+      tmem_wait_st();
+    }
+    tc_fence_before();
+    mbar_arrive(bar(Lay::kBarXchg));
+    if (!wait(bar(Lay::kBarXchg), si & 1)) { ok = false; break; }
+    tc_fence_after();
+    float m_o, l_o;
+    {
+      float x[32];
+      tmem_ld32(tmem + lane_off + kTmemX + 32u * ((si & 1) * 2 + (1 - w)), x);
+      tmem_wait_ld();
+      m_o = x[0];
+      l_o = x[1];
+    }
+    const float m0 = w == 0 ? m_ref : m_o, l0 = w == 0 ? l_sum : l_o;
+    const float m1 = w == 0 ? m_o : m_ref, l1 = w == 0 ? l_o : l_sum;
+    float M = NEG_INF;
+    if (has0) M = fmaxf(M, m0);
+    if (has1) M = fmaxf(M, m1);
+    const float Mr = (M == NEG_INF) ? 0.f : M;
+    const float a0 = has0 ? ex2_approx(m0 - Mr) : 0.f;
+    const float a1 = has1 ? ex2_approx(m1 - Mr) : 0.f;
+    const float Lt = a0 * l0 + a1 * l1;
+    const float inv = (Lt > 0.f) ? 1.f / Lt : 0.f;
+    const float s0 = a0 * inv, s1 = a1 * inv;
+    const int g = row - irow * a.G;
+#pragma unroll 1
+    for (int ch = 0; ch < D / 64; ++ch) {
+      const int col = w * (D / 2) + 32 * ch;
+      float o[32];
+#pragma unroll
+      for (int k = 0; k < 32; ++k) o[k] = 0.f;
+      if (has0) {
+        float x[32];
+        tmem_ld32(t_o0 + col, x);
+        tmem_wait_ld();
+#pragma unroll
+        for (int k = 0; k < 32; ++k) o[k] = x[k] * s0;
+      }
+      if (has1) {
+        float x[32];
+        tmem_ld32(t_o1 + col, x);
+        tmem_wait_ld();
+#pragma unroll
+        for (int k = 0; k < 32; ++k) o[k] = fmaf(x[k], s1, o[k]);
+      }
+      if (my_valid) {
+        if (sg.part < 0) {
+          __nv_bfloat16* dst = a.out + ((long long)(row0 + irow) * a.Hq + h * a.G + g) * D + col;
+          uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            d4[k] = make_uint4(pack_bf16x2(o[8 * k + 0], o[8 * k + 1]),
+                               pack_bf16x2(o[8 * k + 2], o[8 * k + 3]),
+                               pack_bf16x2(o[8 * k + 4], o[8 * k + 5]),
+                               pack_bf16x2(o[8 * k + 6], o[8 * k + 7]));
+        } else {
+          float4* d4 = reinterpret_cast<float4*>(a.ws_o + ((long long)sg.part * kTileM + row) * D + col);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) d4[k] = make_float4(o[4 * k], o[4 * k + 1], o[4 * k + 2], o[4 * k + 3]);
+        }
+      }
+    }
+    if (sg.part >= 0 && w == 0 && my_valid)
+      a.ws_lse[(long long)sg.part * kTileM + row] = M + log2f(Lt);
+    tc_fence_before();
+    mbar_arrive(bar(Lay::kBarOFree));
+    (void)b;
+    ++si;
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kAttnThreads, 1)
+    block_attn_kernel(const __grid_constant__ CUtensorMap tm_q,
+                      const __grid_constant__ CUtensorMap tm_kc,
+                      const __grid_constant__ CUtensorMap tm_vc,
+                      const __grid_constant__ CUtensorMap tm_kb,
+                      const __grid_constant__ CUtensorMap tm_vb, const AttnArgs a) {
+  using Lay = AttnLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kMiscOff);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::kMiscOff + 4);
+  const int warp = threadIdx.x >> 5;
+
+  // A CTA whose range is empty has nothing to set up.
+  {
+    SegCursor cur;
+    cursor_init(a, blockIdx.x, cur);
+    if (cur.remaining <= 0 || cur.b >= a.B) return;
+  }
+
+  if (threadIdx.x == 0) {
+    const uint32_t bars = smem_u32(smem) + Lay::kBarOff;
+    for (int s = 0; s < Lay::kStages; ++s) {
+      mbar_init(bars + 8u * (Lay::kBarKvFull + s), 1);
+      mbar_init(bars + 8u * (Lay::kBarKvEmpty + s), 1);
+    }
+    mbar_init(bars + 8u * Lay::kBarQFull, 1);
+    mbar_init(bars + 8u * Lay::kBarQEmpty, 1);
+    for (int w = 0; w < 2; ++w) {
+      mbar_init(bars + 8u * (Lay::kBarSFull + w), 1);
+      mbar_init(bars + 8u * (Lay::kBarPReady + w), 128);
+      mbar_init(bars + 8u * (Lay::kBarOReady + w), 1);
+    }
+    mbar_init(bars + 8u * Lay::kBarOFree, 256);
+    mbar_init(bars + 8u * Lay::kBarXchg, 256);
+    mbar_init(bars + 8u * Lay::kBarDrain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kProducerWarp && (threadIdx.x & 31) == 0) {
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_kc);
+    prefetch_tmap(&tm_vc);
+    prefetch_tmap(&tm_kb);
+    prefetch_tmap(&tm_vb);
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == kProducerWarp) {
+    if ((threadIdx.x & 31) == 0)
+      producer_role<D>(a, smem, &tm_q, &tm_kc, &tm_vc, &tm_kb, &tm_vb, abort_flag);
+  } else if (warp == kMmaWarp) {
+    mma_role<D>(a, smem, tmem, abort_flag);
+  } else {
+    softmax_role<D>(a, smem, tmem, abort_flag);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
+  if (threadIdx.x == 0 && *abort_flag) raise_flag(a, ORTHRUS_FLAG_TIMEOUT);
+}
+
+// ---------------------------------------------------------------------------
+// Combine: merge the partials of every unit that was cut across CTAs.
+// grid = (B * Hkv, 128 / kCombineRows); 32 threads per query row.
+
+constexpr int kCombineRows = 8;
+
+__device__ __forceinline__ int cta_of_tile(long long T, int C, long long t) {
+  long long c = ((t + 1) * C - 1) / T;
+  if (c > C - 1) c = C - 1;
+  while (c > 0 && range_begin(T, (int)c, C) > t) --c;
+  while (c + 1 < C && range_begin(T, (int)c + 1, C) <= t) ++c;
+  return (int)c;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kCombineRows * 32)
+    attn_combine_kernel(const AttnArgs a) {
+  const int u = blockIdx.x;
+  const int b = u / a.Hkv, h = u % a.Hkv;
+  if (u == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
+    for (int bb = 0; bb < a.B; ++bb)
+      if (seq_rows_bad(a, bb) || seq_len_bad(a, bb)) raise_flag(a, ORTHRUS_FLAG_BAD_LENGTH);
+  }
+  const int Kb = seq_block_len(a, b);
+  if (b >= a.B || Kb <= 0) return;
+  const int nt = seq_tiles(a, b);
+  const int r = blockIdx.y * kCombineRows + (threadIdx.x >> 5);
+  if (r >= a.G * Kb) return;
+  const int lane = threadIdx.x & 31;
+  constexpr int kPer = D / 32;  // elements per thread
+
+  // Partials of this unit: parts p_lo.. in chunked mode, the CTAs of the
+  // covering range (empty CTAs skipped) in balanced mode.
+  int n_parts = 0;
+  int c_lo = 0, c_hi = -1;
+  long long T = 0, s_u = 0;
+  if (a.chunked) {
+    n_parts = unit_chunks(a, nt);
+    if (n_parts <= 1) return;
+  } else {
+    T = total_tiles(a);
+    for (int bb = 0; bb < b; ++bb) s_u += (long long)a.Hkv * seq_tiles(a, bb);
+    s_u += (long long)h * nt;
+    c_lo = cta_of_tile(T, a.num_ctas, s_u);
+    c_hi = cta_of_tile(T, a.num_ctas, s_u + nt - 1);
+    if (c_lo == c_hi) return;
+  }
+  auto part_of = [&](int k, bool& use) -> int {
+    if (a.chunked) {
+      use = true;
+      return u * a.max_chunks + k;
+    }
+    const int cc = c_lo + k;
+    use = range_begin(T, cc, a.num_ctas) < range_begin(T, cc + 1, a.num_ctas);
+    const int slot = (cc == c_lo && s_u > range_begin(T, cc, a.num_ctas)) ? 1 : 0;
+    return cc * 2 + slot;
+  };
+  const int count = a.chunked ? n_parts : (c_hi - c_lo + 1);
+
+  float M = -__int_as_float(0x7f800000);
+  for (int k = 0; k < count; ++k) {
+    bool use;
+    const int p = part_of(k, use);
+    if (use) M = fmaxf(M, a.ws_lse[(long long)p * kTileM + r]);
+  }
+  float acc[kPer];
+#pragma unroll
+  for (int e = 0; e < kPer; ++e) acc[e] = 0.f;
+  float wsum = 0.f;
+  for (int k = 0; k < count; ++k) {
+    bool use;
+    const int p = part_of(k, use);
+    if (!use) continue;
+    const float wgt = exp2f(a.ws_lse[(long long)p * kTileM + r] - M);
+    wsum += wgt;
+    const float* src = a.ws_o + ((long long)p * kTileM + r) * D + lane * kPer;
+#pragma unroll
+    for (int e = 0; e < kPer; e += 2) {
+      const float2 x = *reinterpret_cast<const float2*>(src + e);
+      acc[e] = fmaf(wgt, x.x, acc[e]);
+      acc[e + 1] = fmaf(wgt, x.y, acc[e + 1]);
+    }
+  }
+  const float inv = 1.f / wsum;
+  const int i = r / a.G, g = r - i * a.G;
+  __nv_bfloat16* dst =
+      a.out + ((long long)(seq_row0(a, b) + i) * a.Hq + h * a.G + g) * D + lane * kPer;
+#pragma unroll
+  for (int e = 0; e < kPer; e += 2)
+    *reinterpret_cast<uint32_t*>(dst + e) = pack_bf16x2(acc[e] * inv, acc[e + 1] * inv);
+}
+
+}  // namespace orthrus

@@ -1,0 +1,180 @@
+// Greedy consensus on sm_100a ("Orthrus: Memory-Efficient Parallel Token
+// Generation via Dual-View Diffusion", technical summary §2.3 item 3: accept a
+// drafted token iff it equals the frozen AR view's greedy token, checked left to
+// right; at the first divergence commit the synchronised prefix and the AR
+// correction token).
+//
+// Pass 1 (HBM-bound): every (row, vocabulary chunk) CTA streams its slice of
+// the fp32 logits with 128-bit non-allocating loads and keeps, per thread, the
+// first index of the largest value it has seen (strict >, so NaN never wins and
+// -0 == +0). The winners are packed into 64-bit keys ordered by value, then by
+// lowest index, and max-reduced with warp shuffles into one key per chunk.
+// Pass 2 (tiny): one warp per sequence reduces the chunk keys of its rows,
+// compares each row's greedy token with its draft, finds the first mismatch
+// with a ballot and writes accept length and next token.
+#pragma once
+
+#include <cstdint>
+
+namespace orthrus {
+
+constexpr int kConsThreads = 256;
+constexpr int kConsChunk = 16384;  // logits per CTA in pass 1
+
+// Order-preserving 64-bit key: larger value first, then smaller index.
+// NaN counts as -inf and -0 as +0, so equal keys mean equal values.
+__device__ __forceinline__ unsigned long long consensus_key(float x, uint32_t idx) {
+  uint32_t u = __float_as_uint(x);
+  if (x != x) u = 0xff800000u;          // NaN -> -inf
+  if (u == 0x80000000u) u = 0u;         // -0 -> +0
+  const uint32_t ord = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  return (static_cast<unsigned long long>(ord) << 32) | (0xffffffffu - idx);
+}
+
+__device__ __forceinline__ uint32_t key_index(unsigned long long key) {
+  return 0xffffffffu - static_cast<uint32_t>(key & 0xffffffffull);
+}
+
+__device__ __forceinline__ unsigned long long warp_max_u64(unsigned long long k) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const unsigned long long other = __shfl_xor_sync(0xffffffffu, k, o);
+    k = other > k ? other : k;
+  }
+  return k;
+}
+
+__device__ __forceinline__ float4 ld_nc_f4(const float* p) {
+  float4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "l"(p));
+  return v;
+}
+
+// Keep the first index of the largest value; strict > so ties keep the earlier
+// index and NaN never replaces anything.
+__device__ __forceinline__ void take(float x, int idx, float& best, int& bidx) {
+  if (x > best) {
+    best = x;
+    bidx = idx;
+  }
+}
+
+__global__ void __launch_bounds__(kConsThreads)
+    consensus_argmax_kernel(const float* __restrict__ logits, long long ld, int V,
+                            const int* __restrict__ cu_block, int B, int max_block, int n_chunks,
+                            unsigned long long* __restrict__ part) {
+  const int r = blockIdx.y;
+  const int R = cu_block ? cu_block[B] : B * max_block;
+  if (r >= R) return;
+  const int c = blockIdx.x;
+  const int v0 = c * kConsChunk;
+  const int v1 = min(V, v0 + kConsChunk);
+  const float* row = logits + static_cast<long long>(r) * ld;
+  const int tid = threadIdx.x;
+
+  float best = -__int_as_float(0x7f800000);
+  int bidx = -1;  // -1: this thread saw no element
+  // scalar head up to a 16-byte boundary
+  int head = v0;
+  const int mis = static_cast<int>((reinterpret_cast<uintptr_t>(row + v0) & 15u) >> 2);
+  if (mis) head = min(v1, v0 + (4 - mis));
+  // every thread scans increasing indices, so the first element it sees is its
+  // lowest index: use it as the tie-default when nothing beats -inf
+  if (v0 + tid < head) {
+    bidx = v0 + tid;
+    take(row[v0 + tid], v0 + tid, best, bidx);
+  }
+  const int n4 = (v1 - head) >> 2;
+  const float* vrow = row + head;
+  int i = tid;
+  if (bidx < 0 && i < n4) bidx = head + 4 * i;
+  for (; i + 3 * kConsThreads < n4; i += 4 * kConsThreads) {
+    float4 x[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) x[u] = ld_nc_f4(vrow + 4 * (i + u * kConsThreads));
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int b = head + 4 * (i + u * kConsThreads);
+      take(x[u].x, b, best, bidx);
+      take(x[u].y, b + 1, best, bidx);
+      take(x[u].z, b + 2, best, bidx);
+      take(x[u].w, b + 3, best, bidx);
+    }
+  }
+  for (; i < n4; i += kConsThreads) {
+    const float4 x = ld_nc_f4(vrow + 4 * i);
+    const int b = head + 4 * i;
+    take(x.x, b, best, bidx);
+    take(x.y, b + 1, best, bidx);
+    take(x.z, b + 2, best, bidx);
+    take(x.w, b + 3, best, bidx);
+  }
+  // scalar tail
+  const int tail = head + 4 * n4;
+  if (tail + tid < v1) {
+    if (bidx < 0) bidx = tail + tid;
+    take(row[tail + tid], tail + tid, best, bidx);
+  }
+  unsigned long long key = (bidx >= 0) ? consensus_key(best, static_cast<uint32_t>(bidx)) : 0ull;
+  key = warp_max_u64(key);
+  __shared__ unsigned long long red[kConsThreads / 32];
+  if ((tid & 31) == 0) red[tid >> 5] = key;
+  __syncthreads();
+  if (tid < 32) {
+    key = tid < kConsThreads / 32 ? red[tid] : 0ull;
+    key = warp_max_u64(key);
+    if (tid == 0) part[static_cast<long long>(r) * n_chunks + c] = key;
+  }
+}
+
+__global__ void consensus_finalize_kernel(const unsigned long long* __restrict__ part,
+                                          int n_chunks, const int* __restrict__ draft,
+                                          const int* __restrict__ cu_block, int B, int max_block,
+                                          int* __restrict__ accept_len,
+                                          int* __restrict__ next_token,
+                                          int* __restrict__ row_argmax) {
+  const int warps = blockDim.x >> 5;
+  const int b = blockIdx.x * warps + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (b >= B) return;
+  const int row0 = cu_block ? cu_block[b] : b * max_block;
+  const int Kb = cu_block ? cu_block[b + 1] - row0 : max_block;
+  if (Kb <= 0) {
+    if (lane == 0) {
+      accept_len[b] = 0;
+      next_token[b] = -1;
+    }
+    return;
+  }
+  int m = Kb;  // leading matches
+  int next = -1;
+  for (int base = 0; base < Kb; base += 32) {
+    const int i = base + lane;
+    int t = -1;
+    bool miss = false;
+    if (i < Kb) {
+      unsigned long long k = 0ull;
+      const unsigned long long* p = part + static_cast<long long>(row0 + i) * n_chunks;
+      for (int c = 0; c < n_chunks; ++c) k = p[c] > k ? p[c] : k;
+      t = static_cast<int>(key_index(k));
+      if (row_argmax) row_argmax[row0 + i] = t;
+      miss = draft[row0 + i] != t;
+    }
+    const unsigned ballot = __ballot_sync(0xffffffffu, miss);
+    if (m == Kb && ballot) m = base + __ffs(ballot) - 1;
+    // the committed count is min(m + 1, Kb); its last token lives in this chunk
+    const int n = (m + 1 < Kb) ? (m + 1) : Kb;
+    const int last = n - 1;
+    if (last >= base && last < base + 32 && next < 0) next = __shfl_sync(0xffffffffu, t, last - base);
+    if (m < Kb && !row_argmax) break;
+  }
+  if (lane == 0) {
+    const int n = (m + 1 < Kb) ? (m + 1) : Kb;
+    accept_len[b] = n;
+    next_token[b] = next;
+  }
+}
+
+}  // namespace orthrus

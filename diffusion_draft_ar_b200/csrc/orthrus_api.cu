@@ -1,0 +1,381 @@
+// Host side of the C ABI declared in include/orthrus.h: argument checks (all
+// before any CUDA call), TMA descriptor encoding, launch configuration.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "block_attn.cuh"
+#include "consensus.cuh"
+#include "kv_append.cuh"
+#include "orthrus.h"
+
+namespace {
+
+using namespace orthrus;
+
+thread_local std::string g_last_error;
+
+orthrus_status_t fail(orthrus_status_t s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return s;
+}
+
+orthrus_status_t ok() {
+  g_last_error.clear();
+  return ORTHRUS_OK;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+constexpr int kMaxDevices = 64;
+
+int device_sm_count(int* sms) {
+  static std::atomic<int> cache[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return -1;
+  int v = cache[dev].load(std::memory_order_relaxed);
+  if (v <= 0) {
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
+      return -1;
+    cache[dev].store(v, std::memory_order_relaxed);
+  }
+  *sms = v;
+  return dev;
+}
+
+unsigned long long wait_timeout_ns() {
+  static const unsigned long long v = [] {
+    const char* e = std::getenv("ORTHRUS_WAIT_TIMEOUT_MS");
+    long long ms = e ? std::atoll(e) : 1000;
+    if (ms < 1) ms = 1;
+    return static_cast<unsigned long long>(ms) * 1000000ull;
+  }();
+  return v;
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point, so the
+// library links no driver library and loads on machines without a GPU.
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// bf16 tensor map with 128-byte swizzle; dims/strides innermost first, strides
+// in bytes for dims 1..rank-1.
+bool make_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims,
+              const cuuint64_t* strides, const cuuint32_t* box) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint32_t es[5] = {1, 1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides,
+            box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct AttnPlan {
+  int G, R_max, grid, chunked, chunk_tiles, max_chunks, parts;
+  size_t ws_o_bytes, ws_lse_bytes, ws_bytes;
+};
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Host checks shared by the workspace query and the launch. No CUDA call
+// except the SM-count query (skipped when `sms` is given).
+orthrus_status_t plan_attn(const orthrus_attn_params* p, int sms, AttnPlan* pl) {
+  if (!p) return fail(ORTHRUS_ERR_INVALID_ARG, "params is NULL");
+  if (p->view != ORTHRUS_VIEW_DIFFUSION && p->view != ORTHRUS_VIEW_VERIFY)
+    return fail(ORTHRUS_ERR_INVALID_ARG, "unknown view %d", p->view);
+  if (p->B < 0) return fail(ORTHRUS_ERR_INVALID_ARG, "B = %d < 0", p->B);
+  if (p->Hq < 1 || p->Hkv < 1 || p->Hq % p->Hkv)
+    return fail(ORTHRUS_ERR_INVALID_ARG, "heads Hq = %d, Hkv = %d", p->Hq, p->Hkv);
+  if (p->max_block < 1) return fail(ORTHRUS_ERR_INVALID_ARG, "max_block = %d", p->max_block);
+  if (p->page_size < 1 || p->max_pages_per_seq < 0 || p->num_pages < 0)
+    return fail(ORTHRUS_ERR_INVALID_ARG, "page geometry");
+  if (p->kv_split_tokens < 0 || p->max_ctas < 0)
+    return fail(ORTHRUS_ERR_INVALID_ARG, "kv_split_tokens / max_ctas negative");
+  if (p->D != 64 && p->D != 128) return fail(ORTHRUS_ERR_UNSUPPORTED, "D = %d (64 or 128)", p->D);
+  if (p->page_size % kTileN)
+    return fail(ORTHRUS_ERR_UNSUPPORTED, "page_size = %d (a multiple of 64)", p->page_size);
+  const int G = p->Hq / p->Hkv;
+  if (p->max_block > kTileN || G * p->max_block > kTileM)
+    return fail(ORTHRUS_ERR_UNSUPPORTED, "max_block = %d, G = %d (need K <= 64, G*K <= 128)",
+                p->max_block, G);
+  if (p->kv_split_tokens % kTileN)
+    return fail(ORTHRUS_ERR_UNSUPPORTED, "kv_split_tokens = %d (a multiple of 64)",
+                p->kv_split_tokens);
+  if (static_cast<long long>(p->num_pages) * p->Hkv * p->page_size >= (1ll << 31))
+    return fail(ORTHRUS_ERR_UNSUPPORTED, "cache rows exceed 2^31");
+  if (static_cast<long long>(p->B) * p->max_block >= (1ll << 31) / p->Hq)
+    return fail(ORTHRUS_ERR_UNSUPPORTED, "too many block rows");
+  if (p->total_rows < 0) return fail(ORTHRUS_ERR_INVALID_ARG, "total_rows = %d", p->total_rows);
+  pl->G = G;
+  pl->R_max = p->total_rows > 0 ? p->total_rows : p->B * p->max_block;
+  if (!p->cu_block && pl->R_max < p->B * p->max_block)
+    return fail(ORTHRUS_ERR_INVALID_ARG, "total_rows %d < B * max_block without cu_block",
+                pl->R_max);
+  const long long max_tokens = static_cast<long long>(p->max_pages_per_seq) * p->page_size;
+  if (p->kv_split_tokens > 0) {
+    pl->chunked = 1;
+    pl->chunk_tiles = p->kv_split_tokens / kTileN;
+    const long long ptiles = (max_tokens + kTileN - 1) / kTileN;
+    long long mc = (ptiles + pl->chunk_tiles - 1) / pl->chunk_tiles;
+    if (mc < 1) mc = 1;
+    const long long grid = mc * p->Hkv * static_cast<long long>(p->B);
+    if (grid >= (1ll << 31)) return fail(ORTHRUS_ERR_UNSUPPORTED, "too many chunks");
+    pl->max_chunks = static_cast<int>(mc);
+    pl->grid = static_cast<int>(grid);
+    pl->parts = pl->grid;
+  } else {
+    pl->chunked = 0;
+    pl->chunk_tiles = 0;
+    pl->max_chunks = 0;
+    int c = p->max_ctas > 0 ? p->max_ctas : sms;
+    if (c < 1) c = 1;
+    if (c > 65535) c = 65535;
+    pl->grid = c;
+    pl->parts = 2 * c;
+  }
+  pl->ws_o_bytes = round_up(static_cast<size_t>(pl->parts) * kTileM * p->D * sizeof(float), 256);
+  pl->ws_lse_bytes = round_up(static_cast<size_t>(pl->parts) * kTileM * sizeof(float), 256);
+  pl->ws_bytes = pl->ws_o_bytes + pl->ws_lse_bytes;
+  return ORTHRUS_OK;
+}
+
+template <int D>
+orthrus_status_t launch_attn(const orthrus_attn_params* p, const AttnPlan& pl, int dev,
+                             cudaStream_t stream) {
+  using Lay = AttnLayout<D>;
+  static std::atomic<int> smem_set[kMaxDevices];
+  if (!smem_set[dev].load()) {
+    cudaError_t e = cudaFuncSetAttribute(block_attn_kernel<D>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kAlloc);
+    if (e != cudaSuccess)
+      return fail(ORTHRUS_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    smem_set[dev].store(1);
+  }
+  const int R = pl.R_max;  // rows the caller's block buffers hold
+  CUtensorMap tq, tkc, tvc, tkb, tvb;
+  {
+    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)p->Hq, (cuuint64_t)R};
+    const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)p->Hq * D * 2};
+    const cuuint32_t box[3] = {64, (cuuint32_t)pl.G, (cuuint32_t)std::min(p->max_block, R)};
+    if (!make_map(&tq, p->q_block, 3, dims, strides, box))
+      return fail(ORTHRUS_ERR_CUDA, "tensor map for q_block");
+  }
+  {
+    const cuuint64_t rows = (cuuint64_t)p->num_pages * p->Hkv * p->page_size;
+    const cuuint64_t dims[2] = {(cuuint64_t)D, rows > 0 ? rows : 1};
+    const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+    const cuuint32_t box[2] = {64, (cuuint32_t)kTileN};
+    if (!make_map(&tkc, p->k_cache, 2, dims, strides, box) ||
+        !make_map(&tvc, p->v_cache, 2, dims, strides, box))
+      return fail(ORTHRUS_ERR_CUDA, "tensor map for the KV cache");
+  }
+  {
+    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)p->Hkv, (cuuint64_t)R};
+    const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)p->Hkv * D * 2};
+    const cuuint32_t box[3] = {64, 1, (cuuint32_t)std::min(kTileN, R)};
+    if (!make_map(&tkb, p->k_block, 3, dims, strides, box) ||
+        !make_map(&tvb, p->v_block, 3, dims, strides, box))
+      return fail(ORTHRUS_ERR_CUDA, "tensor map for the block K/V");
+  }
+  AttnArgs a;
+  a.view = p->view;
+  a.B = p->B;
+  a.Hq = p->Hq;
+  a.Hkv = p->Hkv;
+  a.G = pl.G;
+  a.page_size = p->page_size;
+  a.max_pages = p->max_pages_per_seq;
+  a.num_pages = p->num_pages;
+  a.max_block = p->max_block;
+  a.total_rows = pl.R_max;
+  a.prefix_lens = p->prefix_lens;
+  a.cu_block = p->cu_block;
+  a.page_table = p->page_table;
+  a.out = static_cast<__nv_bfloat16*>(p->out);
+  a.ws_o = static_cast<float*>(p->workspace);
+  a.ws_lse = reinterpret_cast<float*>(static_cast<char*>(p->workspace) + pl.ws_o_bytes);
+  a.error_flag = p->error_flag;
+  const float scale = p->softmax_scale > 0.f ? p->softmax_scale : 1.f / std::sqrt((float)D);
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.q_box_rows = std::min(p->max_block, R);
+  a.blk_box_rows = std::min(kTileN, R);
+  a.chunked = pl.chunked;
+  a.chunk_tiles = pl.chunk_tiles;
+  a.max_chunks = pl.max_chunks;
+  a.num_ctas = pl.grid;
+  a.timeout_ns = wait_timeout_ns();
+
+  block_attn_kernel<D><<<pl.grid, kAttnThreads, Lay::kAlloc, stream>>>(tq, tkc, tvc, tkb, tvb, a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(ORTHRUS_ERR_CUDA, "block_attn launch: %s", cudaGetErrorString(e));
+  const int row_groups = (pl.G * p->max_block + kCombineRows - 1) / kCombineRows;
+  dim3 cgrid(p->B * p->Hkv, row_groups);
+  attn_combine_kernel<D><<<cgrid, kCombineRows * 32, 0, stream>>>(a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(ORTHRUS_ERR_CUDA, "combine launch: %s", cudaGetErrorString(e));
+  return ok();
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t orthrus_block_attn_workspace_size(const orthrus_attn_params* p) {
+  int sms = 0;
+  if (!p) return 0;
+  if (p->kv_split_tokens == 0 && p->max_ctas == 0 && device_sm_count(&sms) < 0) return 0;
+  AttnPlan pl;
+  if (plan_attn(p, sms, &pl) != ORTHRUS_OK) return 0;
+  return pl.ws_bytes;
+}
+
+orthrus_status_t orthrus_block_attn(const orthrus_attn_params* p, void* stream) {
+  AttnPlan pl;
+  orthrus_status_t s = plan_attn(p, 1, &pl);  // geometry checks first, no CUDA call
+  if (s != ORTHRUS_OK) return s;
+  if (p->B == 0) return ok();
+  const void* ptrs[] = {p->q_block, p->k_cache, p->v_cache, p->k_block,
+                        p->v_block, p->out,     p->workspace};
+  const char* names[] = {"q_block", "k_cache", "v_cache", "k_block", "v_block", "out", "workspace"};
+  for (int i = 0; i < 7; ++i) {
+    if (!ptrs[i]) return fail(ORTHRUS_ERR_INVALID_ARG, "%s is NULL", names[i]);
+    if (!aligned(ptrs[i], 16)) return fail(ORTHRUS_ERR_INVALID_ARG, "%s is not 16-byte aligned", names[i]);
+  }
+  if (!p->prefix_lens || !p->page_table)
+    return fail(ORTHRUS_ERR_INVALID_ARG, "prefix_lens / page_table is NULL");
+  if (p->max_pages_per_seq < 1 || p->num_pages < 1)
+    return fail(ORTHRUS_ERR_INVALID_ARG, "empty page table or cache");
+  int sms = 0;
+  int dev = 0;
+  if (p->kv_split_tokens == 0 && p->max_ctas == 0) {
+    dev = device_sm_count(&sms);
+    if (dev < 0) return fail(ORTHRUS_ERR_CUDA, "no current CUDA device");
+  } else {
+    if (cudaGetDevice(&dev) != cudaSuccess || dev >= kMaxDevices)
+      return fail(ORTHRUS_ERR_CUDA, "no current CUDA device");
+    sms = 1;
+  }
+  s = plan_attn(p, sms, &pl);
+  if (s != ORTHRUS_OK) return s;
+  if (p->workspace_bytes < pl.ws_bytes)
+    return fail(ORTHRUS_ERR_INVALID_ARG, "workspace %zu bytes < %zu needed", p->workspace_bytes,
+                pl.ws_bytes);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return p->D == 128 ? launch_attn<128>(p, pl, dev, st) : launch_attn<64>(p, pl, dev, st);
+}
+
+size_t orthrus_consensus_workspace_size(int32_t B, int32_t max_block, int32_t V) {
+  if (B < 0 || max_block < 1 || V < 1) return 0;
+  const long long chunks = (V + kConsChunk - 1) / kConsChunk;
+  return static_cast<size_t>(B) * max_block * chunks * sizeof(unsigned long long);
+}
+
+orthrus_status_t orthrus_consensus(const float* verify_logits, int64_t ld, int32_t V,
+                                   const int32_t* draft_tokens, const int32_t* cu_block,
+                                   int32_t B, int32_t max_block, int32_t* accept_len,
+                                   int32_t* next_token, int32_t* row_argmax, void* workspace,
+                                   size_t workspace_bytes, void* stream) {
+  if (B < 0) return fail(ORTHRUS_ERR_INVALID_ARG, "B = %d < 0", B);
+  if (V < 1 || ld < V) return fail(ORTHRUS_ERR_INVALID_ARG, "V = %d, ld = %lld", V, (long long)ld);
+  if (max_block < 1) return fail(ORTHRUS_ERR_INVALID_ARG, "max_block = %d", max_block);
+  if (B == 0) return ok();
+  if (!verify_logits || !draft_tokens || !accept_len || !next_token || !workspace)
+    return fail(ORTHRUS_ERR_INVALID_ARG, "a required pointer is NULL");
+  if (!aligned(verify_logits, 4) || !aligned(workspace, 16))
+    return fail(ORTHRUS_ERR_INVALID_ARG, "misaligned logits or workspace");
+  const long long R_max = static_cast<long long>(B) * max_block;
+  if (R_max >= (1ll << 31)) return fail(ORTHRUS_ERR_UNSUPPORTED, "too many rows");
+  const size_t need = orthrus_consensus_workspace_size(B, max_block, V);
+  if (workspace_bytes < need)
+    return fail(ORTHRUS_ERR_INVALID_ARG, "workspace %zu bytes < %zu needed", workspace_bytes, need);
+  const int n_chunks = (V + kConsChunk - 1) / kConsChunk;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  auto* part = static_cast<unsigned long long*>(workspace);
+  dim3 grid(n_chunks, static_cast<unsigned>(R_max));
+  if (R_max > 65535) return fail(ORTHRUS_ERR_UNSUPPORTED, "more than 65535 rows");
+  consensus_argmax_kernel<<<grid, kConsThreads, 0, st>>>(verify_logits, ld, V, cu_block, B,
+                                                          max_block, n_chunks, part);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(ORTHRUS_ERR_CUDA, "consensus launch: %s", cudaGetErrorString(e));
+  const int warps = 8;
+  consensus_finalize_kernel<<<(B + warps - 1) / warps, warps * 32, 0, st>>>(
+      part, n_chunks, draft_tokens, cu_block, B, max_block, accept_len, next_token, row_argmax);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(ORTHRUS_ERR_CUDA, "consensus launch: %s", cudaGetErrorString(e));
+  return ok();
+}
+
+orthrus_status_t orthrus_kv_append(const void* k_block, const void* v_block,
+                                   const int32_t* cu_block, int32_t max_block,
+                                   const int32_t* accept_len, int32_t* prefix_lens,
+                                   int32_t update_lens, const int32_t* page_table,
+                                   int32_t max_pages_per_seq, int32_t num_pages, void* k_cache,
+                                   void* v_cache, int32_t B, int32_t Hkv, int32_t D,
+                                   int32_t page_size, int32_t* error_flag, void* stream) {
+  if (B < 0 || Hkv < 1 || D < 8 || D % 8 || page_size < 1 || max_pages_per_seq < 0 ||
+      num_pages < 0 || (!cu_block && max_block < 1))
+    return fail(ORTHRUS_ERR_INVALID_ARG, "bad sizes (B %d, Hkv %d, D %d, P %d)", B, Hkv, D,
+                page_size);
+  if (B == 0) return ok();
+  if (!k_block || !v_block || !accept_len || !prefix_lens || !page_table || !k_cache || !v_cache)
+    return fail(ORTHRUS_ERR_INVALID_ARG, "a required pointer is NULL");
+  if (!aligned(k_block, 16) || !aligned(v_block, 16) || !aligned(k_cache, 16) ||
+      !aligned(v_cache, 16))
+    return fail(ORTHRUS_ERR_INVALID_ARG, "K/V pointers must be 16-byte aligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  kv_append_kernel<<<B, kAppendThreads, 0, st>>>(
+      static_cast<const uint4*>(k_block), static_cast<const uint4*>(v_block), cu_block, max_block,
+      accept_len, prefix_lens, update_lens, page_table, max_pages_per_seq, num_pages,
+      static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), Hkv, D, page_size, error_flag);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(ORTHRUS_ERR_CUDA, "kv_append launch: %s", cudaGetErrorString(e));
+  return ok();
+}
+
+const char* orthrus_status_string(orthrus_status_t s) {
+  switch (s) {
+    case ORTHRUS_OK: return "ok";
+    case ORTHRUS_ERR_INVALID_ARG: return "invalid argument";
+    case ORTHRUS_ERR_UNSUPPORTED: return "unsupported configuration";
+    case ORTHRUS_ERR_CUDA: return "CUDA error";
+    case ORTHRUS_ERR_TIMEOUT: return "device wait timed out";
+    case ORTHRUS_ERR_DEVICE_CHECK: return "device-side check failed";
+  }
+  return "unknown status";
+}
+
+const char* orthrus_last_error(void) { return g_last_error.c_str(); }
+
+int32_t orthrus_abi_version(void) { return ORTHRUS_ABI_VERSION; }
+
+}  // extern "C"

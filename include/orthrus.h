@@ -1,0 +1,211 @@
+/*
+ * orthrus.h -- C ABI of the Orthrus block-decoding hot path on NVIDIA B200 (sm_100a).
+ *
+ * Orthrus ("Orthrus: Memory-Efficient Parallel Token Generation via Dual-View
+ * Diffusion") lets a lightweight diffusion view draft a block of K tokens (the
+ * anchor plus K-1 mask slots) over the KV cache that a frozen autoregressive
+ * (AR) view built, then has the AR view verify the whole block in one pass and
+ * keeps the drafts that equal the AR greedy tokens. This library implements the
+ * three data-parallel steps of one round:
+ *
+ *   orthrus_block_attn  attention of the block rows over the shared paged prefix
+ *                       cache plus the block's own K/V, in the DIFFUSION view
+ *                       (bidirectional inside the block) or the VERIFY view
+ *                       (causal inside the block);
+ *   orthrus_consensus   greedy argmax of the verify logits and the left-to-right
+ *                       exact match against the drafts;
+ *   orthrus_kv_append   commit: write the accepted rows' K/V into the cache.
+ *
+ * Conventions shared by every call:
+ *   - Every pointer marked "device" is a device pointer owned by the caller; the
+ *     library never allocates, frees or retains memory and keeps no per-call
+ *     state (it caches TMA descriptors' driver entry point and device
+ *     attributes only).
+ *   - `stream` is a cudaStream_t passed as an opaque pointer (NULL = the legacy
+ *     default stream). Every call is asynchronous on it.
+ *   - Arguments are checked on the host before anything is launched; a failed
+ *     check returns ORTHRUS_ERR_INVALID_ARG or ORTHRUS_ERR_UNSUPPORTED and
+ *     launches nothing. A failed launch returns ORTHRUS_ERR_CUDA.
+ *   - Data that can only be checked on the device (a page index out of range, a
+ *     length beyond the page table, a pipeline wait that ran out of time) is
+ *     reported by OR-ing ORTHRUS_FLAG_* bits into the optional device word
+ *     `error_flag`; the offending work item skips its writes. No kernel traps.
+ *   - bf16 is IEEE binary32's upper 16 bits; all layouts are row-major and
+ *     densely packed.
+ *   - Outputs must not alias inputs.
+ */
+#ifndef ORTHRUS_H_
+#define ORTHRUS_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define ORTHRUS_ABI_VERSION 1
+
+#if defined(ORTHRUS_BUILD) && defined(__GNUC__)
+#define ORTHRUS_API __attribute__((visibility("default")))
+#else
+#define ORTHRUS_API
+#endif
+
+typedef enum {
+  ORTHRUS_OK = 0,
+  ORTHRUS_ERR_INVALID_ARG = 1,  /* a pointer, size or layout argument is wrong */
+  ORTHRUS_ERR_UNSUPPORTED = 2,  /* valid, but outside what the kernels implement */
+  ORTHRUS_ERR_CUDA = 3,         /* the CUDA runtime refused a launch or query */
+  ORTHRUS_ERR_TIMEOUT = 4,      /* reserved for callers mapping ORTHRUS_FLAG_TIMEOUT */
+  ORTHRUS_ERR_DEVICE_CHECK = 5  /* reserved for callers mapping the other flag bits */
+} orthrus_status_t;
+
+/* Bits OR-ed into *error_flag by the kernels. */
+#define ORTHRUS_FLAG_BAD_PAGE 0x1   /* a page_table entry was outside [0, num_pages) */
+#define ORTHRUS_FLAG_BAD_LENGTH 0x2 /* prefix_len + rows ran past max_pages_per_seq pages,
+                                       or accept_len outside [0, K_b] */
+#define ORTHRUS_FLAG_TIMEOUT 0x4    /* a pipeline wait gave up; that CTA wrote nothing */
+
+typedef enum {
+  ORTHRUS_VIEW_DIFFUSION = 0, /* block rows see the whole prefix and every block row */
+  ORTHRUS_VIEW_VERIFY = 1     /* block row i sees the whole prefix and block rows 0..i */
+} orthrus_view_t;
+
+/*
+ * Parameters of orthrus_block_attn.
+ *
+ * Operation (technical summary §2.2 "attention mechanism", mask M_diff, for the
+ * DIFFUSION view; §2.3 item 2, the AR view's single-pass check of the populated
+ * block, for the VERIFY view). For every sequence b, KV head h, block row i in
+ * [0, K_b) and query head hq = h*G + g (G = Hq / Hkv, g in [0, G)):
+ *
+ *   out[row0_b + i, hq, :] = sum_j softmax_j(scale * <q, k_j>) * v_j
+ *
+ * with q = q_block[row0_b + i, hq, :] and j running over the visible keys: the
+ * prefix positions t in [0, L_b) (k_j = k_cache[page_table[b][t / P], h, t % P, :])
+ * followed by the block rows j' in [0, K_b) (k_j = k_block[row0_b + j', h, :]),
+ * block row j' being visible to row i always (DIFFUSION) or iff j' <= i (VERIFY).
+ * L_b = prefix_lens[b]; row0_b = cu_block[b]; K_b = cu_block[b+1] - cu_block[b].
+ * The same indexing gives v_j. Accumulation is fp32, the output is rounded to bf16.
+ *
+ * Work is split over the prefix (split-KV): each CTA covers a contiguous range
+ * of 64-token tiles and writes either the final rows or a partial (row max, sum,
+ * normalised accumulator) that a combine kernel merges.
+ */
+typedef struct {
+  int32_t view;              /* orthrus_view_t */
+  int32_t B;                 /* sequences, >= 0 (0: nothing to do) */
+  int32_t Hq, Hkv;           /* query / KV heads; Hq % Hkv == 0 */
+  int32_t D;                 /* head dim: 64 or 128 */
+  int32_t page_size;         /* tokens per page P: a multiple of 64 */
+  int32_t max_pages_per_seq; /* columns of page_table */
+  int32_t num_pages;         /* pages in k_cache / v_cache */
+  int32_t max_block;         /* max K_b: 1..64 and G * max_block <= 128 */
+  int32_t total_rows;        /* R, rows of q_block, k_block, v_block and out; cu_block[B]
+                                must not exceed it (0: R = B * max_block) */
+  const void* q_block;       /* device bf16 [R, Hq, D] */
+  const void* k_cache;       /* device bf16 [num_pages, Hkv, P, D] */
+  const void* v_cache;       /* device bf16 [num_pages, Hkv, P, D] */
+  const void* k_block;       /* device bf16 [R, Hkv, D] */
+  const void* v_block;       /* device bf16 [R, Hkv, D] */
+  const int32_t* prefix_lens; /* device [B] */
+  const int32_t* cu_block;   /* device [B+1] row offsets; NULL: every K_b = max_block */
+  const int32_t* page_table; /* device [B, max_pages_per_seq] */
+  float softmax_scale;       /* <= 0: 1/sqrt(D) */
+  int32_t kv_split_tokens;   /* 0: balanced split over the SMs; > 0: fixed chunks of this
+                                many prefix tokens (a multiple of 64), one CTA each */
+  int32_t max_ctas;          /* 0: one CTA per SM; > 0: cap for the balanced split */
+  void* out;                 /* device bf16 [R, Hq, D] */
+  void* workspace;           /* device scratch, >= orthrus_block_attn_workspace_size() bytes,
+                                256-byte aligned; contents need no initialisation */
+  size_t workspace_bytes;
+  int32_t* error_flag;       /* optional device int32; ORTHRUS_FLAG_* bits are OR-ed in */
+} orthrus_attn_params;
+
+/* Scratch bytes orthrus_block_attn needs for these parameters (queries the
+ * current device's SM count). 0 when the parameters are invalid. */
+ORTHRUS_API size_t orthrus_block_attn_workspace_size(const orthrus_attn_params* p);
+
+/* Launch the block attention described by *p on `stream`.
+ * q_block, k_block, v_block and out hold total_rows rows; a sequence whose
+ * cu_block range is decreasing, longer than max_block or past total_rows is
+ * skipped and flagged (ORTHRUS_FLAG_BAD_LENGTH). All device pointers 16-byte
+ * aligned. Errors: INVALID_ARG (null pointer, bad sizes, misalignment, short
+ * workspace), UNSUPPORTED (D, page_size, max_block or G*max_block outside the
+ * implemented set), CUDA (launch failure). */
+ORTHRUS_API orthrus_status_t orthrus_block_attn(const orthrus_attn_params* p, void* stream);
+
+/*
+ * Greedy consensus (technical summary §2.3 item 3: a drafted token is accepted
+ * iff it equals the frozen AR view's greedy token, checked left to right; at the
+ * first divergence j the prefix up to j-1 is committed and the exact AR
+ * correction token appended; agents-report.net commentary, "core design").
+ *
+ * For every block row r: t_r = argmax_v verify_logits[r, v] (the lowest index
+ * among equal maxima; NaN counts as -inf; -0 == +0). For every sequence b with
+ * K_b > 0: m_b = number of leading rows r = row0_b + i with draft_tokens[r] ==
+ * t_r; accept_len[b] = min(m_b + 1, K_b); next_token[b] = t_{row0_b +
+ * accept_len[b] - 1}. A sequence with K_b = 0 gets accept_len 0, next_token -1.
+ *
+ *   verify_logits  device fp32 [R, ld] (row r at verify_logits + r*ld), V <= ld
+ *   draft_tokens   device int32 [R]
+ *   cu_block       device int32 [B+1] or NULL (every K_b = max_block)
+ *   accept_len, next_token  device int32 [B] (written)
+ *   row_argmax     device int32 [R] or NULL (written when given)
+ *   workspace      device scratch of orthrus_consensus_workspace_size(B, max_block, V)
+ *                  bytes, 16-byte aligned; contents need no initialisation
+ * R = cu_block[B] <= B * max_block. Errors: INVALID_ARG, CUDA.
+ */
+ORTHRUS_API size_t orthrus_consensus_workspace_size(int32_t B, int32_t max_block, int32_t V);
+ORTHRUS_API orthrus_status_t orthrus_consensus(const float* verify_logits, int64_t ld, int32_t V,
+                                   const int32_t* draft_tokens, const int32_t* cu_block,
+                                   int32_t B, int32_t max_block, int32_t* accept_len,
+                                   int32_t* next_token, int32_t* row_argmax, void* workspace,
+                                   size_t workspace_bytes, void* stream);
+
+/*
+ * Commit (technical summary §2.3 item 3, commit the synchronised prefix and
+ * truncate the cache; agents-report.net commentary, "core design", the accepted
+ * tokens' KV appended to the shared cache). For every sequence b, accepted row
+ * i in [0, accept_len[b]) and KV head h, with L_b = prefix_lens[b] on entry:
+ *
+ *   k_cache[page_table[b][(L_b+i)/P], h, (L_b+i) % P, :] = k_block[cu_block[b]+i, h, :]
+ *
+ * and the same for V; no other cache byte is written. With update_lens != 0,
+ * prefix_lens[b] becomes L_b + accept_len[b] (only when every row of b found its
+ * page; otherwise ORTHRUS_FLAG_* is raised and b's length is left unchanged).
+ *
+ *   k_block, v_block  device bf16 [R, Hkv, D] (the VERIFY view's block K/V)
+ *   cu_block          device int32 [B+1], or NULL: every block has max_block rows
+ *                     (row0_b = b * max_block)
+ *   accept_len        device int32 [B]
+ *   prefix_lens       device int32 [B] (read; updated in place iff update_lens)
+ *   page_table        device int32 [B, max_pages_per_seq]
+ *   k_cache, v_cache  device bf16 [num_pages, Hkv, page_size, D] (updated in place)
+ *   error_flag        optional device int32
+ * D must be a multiple of 8 and the pointers 16-byte aligned. Errors:
+ * INVALID_ARG, CUDA.
+ */
+ORTHRUS_API orthrus_status_t orthrus_kv_append(const void* k_block, const void* v_block,
+                                   const int32_t* cu_block, int32_t max_block,
+                                   const int32_t* accept_len, int32_t* prefix_lens,
+                                   int32_t update_lens, const int32_t* page_table,
+                                   int32_t max_pages_per_seq, int32_t num_pages, void* k_cache,
+                                   void* v_cache, int32_t B, int32_t Hkv, int32_t D,
+                                   int32_t page_size, int32_t* error_flag, void* stream);
+
+/* Static description of a status code. */
+ORTHRUS_API const char* orthrus_status_string(orthrus_status_t status);
+
+/* Detail of the last failed call on this host thread ("" when none). */
+ORTHRUS_API const char* orthrus_last_error(void);
+
+/* ORTHRUS_ABI_VERSION of the loaded library. */
+ORTHRUS_API int32_t orthrus_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ORTHRUS_H_ */

@@ -1,0 +1,150 @@
+"""The C-ABI library without a GPU: it loads, exports every symbol the header
+declares, its parameter struct matches the header's layout, and bad arguments
+are refused on the host before anything touches CUDA."""
+import ctypes
+import os
+import re
+import subprocess
+import tempfile
+
+import pytest
+
+from diffusion_draft_ar_b200 import build as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "orthrus.h")
+
+
+@pytest.fixture(scope="module")
+def O():
+    B.build()
+    from diffusion_draft_ar_b200 import orthrus
+    return orthrus
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    return re.findall(r"^ORTHRUS_API\s+[\w\s\*]+?\b(orthrus_\w+)\s*\(", src, flags=re.M)
+
+
+def test_every_declared_symbol_is_exported(O):
+    names = declared_functions()
+    assert set(names) >= {"orthrus_block_attn", "orthrus_block_attn_workspace_size",
+                          "orthrus_consensus", "orthrus_consensus_workspace_size",
+                          "orthrus_kv_append", "orthrus_status_string", "orthrus_last_error",
+                          "orthrus_abi_version"}
+    out = subprocess.run(["nm", "-D", "--defined-only", B.LIB], capture_output=True, text=True,
+                         check=True).stdout
+    exported = {l.split()[-1] for l in out.splitlines() if " T " in l}
+    for n in names:
+        assert n in exported, n
+        assert hasattr(O.lib, n)
+    # nothing else leaks out of the library under an orthrus_ name
+    assert {n for n in exported if n.startswith("orthrus_")} == set(names)
+
+
+def test_abi_version_and_status_strings(O):
+    assert O.abi_version() == 1
+    for s in range(6):
+        assert O.lib.orthrus_status_string(s)
+    assert O.lib.orthrus_status_string(99) == b"unknown status"
+
+
+def test_param_struct_layout_matches_header(O):
+    fields = [f[0] for f in O.AttnParams._fields_]
+    prog = ["#include <stdio.h>", "#include <stddef.h>", '#include "orthrus.h"', "int main(void){",
+            'printf("%zu\\n", sizeof(orthrus_attn_params));']
+    for f in fields:
+        prog.append(f'printf("%zu\\n", offsetof(orthrus_attn_params, {f}));')
+    prog.append("return 0;}")
+    with tempfile.TemporaryDirectory() as d:
+        c = os.path.join(d, "layout.c")
+        exe = os.path.join(d, "layout")
+        open(c, "w").write("\n".join(prog))
+        subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), "-o", exe, c], check=True)
+        vals = [int(x) for x in subprocess.run([exe], capture_output=True, text=True,
+                                                check=True).stdout.split()]
+    assert vals[0] == ctypes.sizeof(O.AttnParams)
+    for f, off in zip(fields, vals[1:]):
+        assert getattr(O.AttnParams, f).offset == off, f
+
+
+def _params(O, **kw):
+    p = O.AttnParams()
+    base = dict(view=1, B=2, Hq=8, Hkv=2, D=128, page_size=64, max_pages_per_seq=4, num_pages=8,
+                max_block=8, total_rows=16, q_block=0x10000, k_cache=0x20000, v_cache=0x30000,
+                k_block=0x40000, v_block=0x50000, prefix_lens=0x60000, cu_block=None,
+                page_table=0x70000, softmax_scale=0.0, kv_split_tokens=0, max_ctas=0,
+                out=0x80000, workspace=0x90000, workspace_bytes=1 << 30, error_flag=None)
+    base.update(kw)
+    for k, v in base.items():
+        setattr(p, k, v)
+    return p
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(view=2), 1), (dict(B=-1), 1), (dict(Hq=6, Hkv=4), 1), (dict(Hkv=0), 1),
+    (dict(max_block=0), 1), (dict(D=96), 2), (dict(page_size=32), 2), (dict(max_block=65), 2),
+    (dict(Hq=16, Hkv=1, max_block=16), 2), (dict(kv_split_tokens=100), 2),
+    (dict(kv_split_tokens=-64), 1), (dict(total_rows=-1), 1), (dict(total_rows=4), 1),
+    (dict(q_block=None), 1), (dict(out=None), 1), (dict(k_cache=0x20008), 1),
+    (dict(workspace=None), 1), (dict(prefix_lens=None), 1), (dict(page_table=None), 1),
+    (dict(num_pages=0), 1), (dict(max_pages_per_seq=0), 1),
+])
+def test_block_attn_rejects_bad_arguments(O, kw, status):
+    p = _params(O, **kw)
+    assert O.lib.orthrus_block_attn(ctypes.byref(p), None) == status
+    assert O.lib.orthrus_last_error() != b""
+
+
+def test_block_attn_empty_batch_is_a_no_op(O):
+    p = _params(O, B=0, q_block=None, out=None)
+    assert O.lib.orthrus_block_attn(ctypes.byref(p), None) == 0
+
+
+def test_block_attn_workspace_size_chunked_mode(O):
+    # fixed 2048-token chunks: one partial per CTA, grid = chunks * Hkv * B
+    p = _params(O, B=1, Hq=32, Hkv=8, max_block=32, total_rows=32, max_pages_per_seq=2049,
+                num_pages=2049, kv_split_tokens=2048)
+    n = O.block_attn_workspace_size(p)
+    chunks = -(-2049 * 64 // 2048)
+    parts = chunks * 8
+    assert n == parts * 128 * 128 * 4 + (-(-parts * 128 * 4 // 256)) * 256
+    assert O.block_attn_workspace_size(_params(O, D=96, kv_split_tokens=64)) == 0
+
+
+@pytest.mark.parametrize("args,status", [
+    (dict(V=0), 1), (dict(ld=10, V=20), 1), (dict(B=-1), 1), (dict(max_block=0), 1),
+    (dict(logits=None), 1), (dict(draft=None), 1), (dict(workspace=None), 1),
+    (dict(workspace_bytes=8), 1), (dict(logits=0x10002), 1),
+])
+def test_consensus_rejects_bad_arguments(O, args, status):
+    a = dict(logits=0x10000, ld=512, V=512, draft=0x20000, cu=None, B=2, max_block=8,
+             acc=0x30000, nxt=0x40000, am=None, workspace=0x50000, workspace_bytes=1 << 20)
+    a.update(args)
+    st = O.lib.orthrus_consensus(a["logits"], a["ld"], a["V"], a["draft"], a["cu"], a["B"],
+                                 a["max_block"], a["acc"], a["nxt"], a["am"], a["workspace"],
+                                 a["workspace_bytes"], None)
+    assert st == status
+
+
+def test_consensus_workspace_size(O):
+    assert O.consensus_workspace_size(16, 32, 151936) == 16 * 32 * 10 * 8
+    assert O.consensus_workspace_size(1, 8, 512) == 8 * 8
+    assert O.consensus_workspace_size(-1, 8, 512) == 0
+
+
+@pytest.mark.parametrize("args", [
+    dict(D=12), dict(Hkv=0), dict(page_size=0), dict(k_block=None), dict(prefix_lens=None),
+    dict(k_cache=0x30004), dict(cu=None, max_block=0),
+])
+def test_kv_append_rejects_bad_arguments(O, args):
+    a = dict(k_block=0x10000, v_block=0x20000, cu=0x1000, max_block=8, acc=0x2000, lens=0x3000,
+             table=0x4000, k_cache=0x30000, v_cache=0x40000, B=2, Hkv=2, D=128, page_size=64)
+    if "prefix_lens" in args:
+        a["lens"] = args.pop("prefix_lens")
+    a.update(args)
+    st = O.lib.orthrus_kv_append(a["k_block"], a["v_block"], a["cu"], a["max_block"], a["acc"],
+                                 a["lens"], 1, a["table"], 4, 8, a["k_cache"], a["v_cache"],
+                                 a["B"], a["Hkv"], a["D"], a["page_size"], None, None)
+    assert st == 1
