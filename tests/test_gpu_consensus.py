@@ -93,7 +93,7 @@ def test_odd_vocab_and_unaligned_rows(V, ld):
     # repeat the row maximum at a later index to check tie handling across chunks
     for r in range(R):
         j = int(buf[r, :V].argmax())
-        buf[r, V - 1 - (r % 3)] = buf[r, j]
+        buf[r, max(0, V - 1 - (r % 3))] = buf[r, j]
     t = buf[:, :V].argmax(1)
     drafts = torch.from_numpy(np.where(g.random(R) < 0.8, t, (t + 1) % V).astype(np.int32))
     cu = torch.tensor([0, 5, 5, 12, 24], dtype=torch.int32)
