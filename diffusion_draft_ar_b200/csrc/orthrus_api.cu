@@ -362,6 +362,82 @@ orthrus_status_t orthrus_kv_append(const void* k_block, const void* v_block,
   return ok();
 }
 
+// ---------------------------------------------------------------------------
+// Consensus for callers that cannot allocate device memory at call time (an
+// engine that pre-reserves all of HBM and hands plug-ins no scratch, or a
+// decode path that must not pay cudaMalloc's implicit synchronisation). The
+// partial keys live in this fixed array instead of a caller workspace.
+
+constexpr long long kNoAllocScratchKeys = 65536;  // 512 KiB of 64-bit keys
+
+static __device__ __align__(256) unsigned long long g_consensus_scratch[kNoAllocScratchKeys];
+
+}  // extern "C"
+
+namespace {
+
+// Device address of g_consensus_scratch on the current device. In host code
+// the array's name is only a host-side stand-in, so the address is looked up
+// once per device (with that device current) and cached.
+unsigned long long* noalloc_scratch(int* dev_out) {
+  static std::mutex mu;
+  static void* addr[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  *dev_out = dev;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_consensus_scratch) != cudaSuccess || !p) return nullptr;
+    addr[dev] = p;
+  }
+  return static_cast<unsigned long long*>(addr[dev]);
+}
+
+}  // namespace
+
+extern "C" {
+
+orthrus_status_t orthrus_consensus_noalloc(const float* verify_logits, int64_t ld, int32_t V,
+                                           const int32_t* draft_tokens, const int32_t* cu_block,
+                                           int32_t B, int32_t max_block, int32_t* accept_len,
+                                           int32_t* next_token, int32_t* row_argmax,
+                                           void* stream) {
+  if (B < 0) return fail(ORTHRUS_ERR_INVALID_ARG, "B = %d < 0", B);
+  if (V < 1 || ld < V) return fail(ORTHRUS_ERR_INVALID_ARG, "V = %d, ld = %lld", V, (long long)ld);
+  if (max_block < 1) return fail(ORTHRUS_ERR_INVALID_ARG, "max_block = %d", max_block);
+  if (B == 0) return ok();
+  if (!verify_logits || !draft_tokens || !accept_len || !next_token)
+    return fail(ORTHRUS_ERR_INVALID_ARG, "a required pointer is NULL");
+  if (!aligned(verify_logits, 4)) return fail(ORTHRUS_ERR_INVALID_ARG, "misaligned logits");
+  const long long n_chunks = (V + kConsChunk - 1) / kConsChunk;
+  const long long R_max = static_cast<long long>(B) * max_block;
+  if (R_max > 65535) return fail(ORTHRUS_ERR_UNSUPPORTED, "more than 65535 rows");
+  const long long keys = R_max * n_chunks;
+  if (keys > kNoAllocScratchKeys)
+    return fail(ORTHRUS_ERR_UNSUPPORTED,
+                "request needs %lld scratch keys (B*max_block*ceil(V/16384)); the built-in "
+                "array holds %lld",
+                keys, kNoAllocScratchKeys);
+  int dev = 0;
+  unsigned long long* part = noalloc_scratch(&dev);
+  if (!part) return fail(ORTHRUS_ERR_CUDA, "cannot resolve the scratch array's device address");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  dim3 grid(static_cast<unsigned>(n_chunks), static_cast<unsigned>(R_max));
+  consensus_argmax_kernel<<<grid, kConsThreads, 0, st>>>(verify_logits, ld, V, cu_block, B,
+                                                          max_block, static_cast<int>(n_chunks),
+                                                          part);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(ORTHRUS_ERR_CUDA, "consensus launch: %s", cudaGetErrorString(e));
+  const int warps = 8;
+  consensus_finalize_kernel<<<(B + warps - 1) / warps, warps * 32, 0, st>>>(
+      part, static_cast<int>(n_chunks), draft_tokens, cu_block, B, max_block, accept_len,
+      next_token, row_argmax);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(ORTHRUS_ERR_CUDA, "consensus launch: %s", cudaGetErrorString(e));
+  return ok();
+}
+
 const char* orthrus_status_string(orthrus_status_t s) {
   switch (s) {
     case ORTHRUS_OK: return "ok";

@@ -57,6 +57,8 @@ lib.orthrus_consensus.argtypes = [_vp, _i64, _i32, _vp, _vp, _i32, _i32, _vp, _v
 lib.orthrus_kv_append.restype = _i32
 lib.orthrus_kv_append.argtypes = [_vp, _vp, _vp, _i32, _vp, _vp, _i32, _vp, _i32, _i32, _vp, _vp,
                                   _i32, _i32, _i32, _i32, _vp, _vp]
+lib.orthrus_consensus_noalloc.restype = _i32
+lib.orthrus_consensus_noalloc.argtypes = [_vp, _i64, _i32, _vp, _vp, _i32, _i32, _vp, _vp, _vp, _vp]
 lib.orthrus_status_string.restype = ctypes.c_char_p
 lib.orthrus_status_string.argtypes = [_i32]
 lib.orthrus_last_error.restype = ctypes.c_char_p
@@ -174,6 +176,29 @@ def consensus(verify_logits, draft_tokens, cu_block, B: int, max_block: int, acc
                                _ptr(next_token), _ptr(row_argmax), _ptr(workspace),
                                workspace.numel(), _stream(stream))
     _check(st, "orthrus_consensus")
+
+
+def consensus_noalloc(verify_logits, draft_tokens, cu_block, B: int, max_block: int, accept_len,
+                      next_token, row_argmax=None, stream=None):
+    """``orthrus_consensus_noalloc``: consensus for callers that cannot hand the
+    library a device workspace (the scratch is a fixed array inside the library;
+    see the header for its size limit and the rule on overlapping calls)."""
+    if not verify_logits.is_cuda or verify_logits.dtype != torch.float32 or verify_logits.dim() != 2:
+        raise ValueError("verify_logits must be a 2-D CUDA float32 tensor")
+    if verify_logits.stride(1) != 1:
+        raise ValueError("verify_logits rows must be contiguous")
+    _need(draft_tokens, "draft_tokens", torch.int32, 1)
+    _need(accept_len, "accept_len", torch.int32, 1)
+    _need(next_token, "next_token", torch.int32, 1)
+    if cu_block is not None:
+        _need(cu_block, "cu_block", torch.int32, 1)
+    if row_argmax is not None:
+        _need(row_argmax, "row_argmax", torch.int32, 1)
+    st = lib.orthrus_consensus_noalloc(_ptr(verify_logits), verify_logits.stride(0),
+                                       verify_logits.shape[1], _ptr(draft_tokens), _ptr(cu_block),
+                                       int(B), int(max_block), _ptr(accept_len), _ptr(next_token),
+                                       _ptr(row_argmax), _stream(stream))
+    _check(st, "orthrus_consensus_noalloc")
 
 
 def kv_append(k_block, v_block, cu_block, max_block: int, accept_len, prefix_lens, page_table,

@@ -195,6 +195,38 @@ ORTHRUS_API orthrus_status_t orthrus_kv_append(const void* k_block, const void* 
                                    void* v_cache, int32_t B, int32_t Hkv, int32_t D,
                                    int32_t page_size, int32_t* error_flag, void* stream);
 
+/*
+ * Greedy consensus without any device allocation (no counterpart in the
+ * paper; it is a deployment convenience of this library).
+ *
+ * Same operation, arguments and results as orthrus_consensus, minus the
+ * workspace. It is meant for callers that cannot allocate device memory when
+ * they call in: a serving engine that reserves every byte of HBM at start-up
+ * and gives its plug-ins no scratch, or a caller that must not trigger the
+ * implicit device synchronisation and latency of cudaMalloc on its decode
+ * path. The scratch lives instead in a fixed 512 KiB array inside the library
+ * (a file-scope __device__ array, so every GPU that loads the library holds it
+ * until the process exits):
+ *   - the request must fit: B * max_block * ceil(V / 16384) <= 65536 (for
+ *     V = 151936 that is B * max_block <= 6553 rows); larger requests return
+ *     ORTHRUS_ERR_UNSUPPORTED and launch nothing;
+ *   - the first call on a device looks up the array's device address for that
+ *     device (a runtime symbol query, no allocation); make that first call
+ *     before any stream capture;
+ *   - every call on a device uses the same array, so calls whose kernels can
+ *     overlap on the GPU (different streams without ordering) race: order them
+ *     on one stream or with events. Nothing in the array needs to start at
+ *     zero: each call writes every slot it later reads.
+ * The call itself allocates nothing (no cudaMalloc, cudaFree or allocating
+ * library routine). Errors: as orthrus_consensus, plus UNSUPPORTED above.
+ */
+ORTHRUS_API orthrus_status_t orthrus_consensus_noalloc(const float* verify_logits, int64_t ld,
+                                                       int32_t V, const int32_t* draft_tokens,
+                                                       const int32_t* cu_block, int32_t B,
+                                                       int32_t max_block, int32_t* accept_len,
+                                                       int32_t* next_token, int32_t* row_argmax,
+                                                       void* stream);
+
 /* Static description of a status code. */
 ORTHRUS_API const char* orthrus_status_string(orthrus_status_t status);
 
