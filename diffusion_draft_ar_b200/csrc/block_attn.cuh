@@ -17,14 +17,19 @@
 // kernel from per-CTA partials (max, sum, normalised accumulator).
 //
 // Roles (320 threads):
-//   warp 0      TMA producer: Q tile per unit, K and V tiles into a ring of
-//               stages, page ids read from the page table.
-//   warp 1      MMA issuer: S = Q K^T into TMEM, then O += P V; owns TMEM.
+//   warp 0      TMA producer: Q tile per unit; K tiles into a K ring and V
+//               tiles into a separate, deeper V ring (K is released by its
+//               QK three tiles before V is released by its PV); the next
+//               page id is fetched while the current tile's copies are issued.
+//   warp 1      MMA issuer: S = Q K^T into one of three TMEM S buffers, running
+//               three tiles ahead of O += P V, so a softmax group never waits
+//               for a QK round trip; owns TMEM.
 //   warps 2-5   softmax group 0 (even tiles), warps 6-9 softmax group 1 (odd
 //               tiles). Each thread owns one query row (= one TMEM lane): it
 //               reads its S row from TMEM, applies the view's mask, keeps a
-//               running max/sum, writes P (bf16) to shared memory for the PV
-//               MMA and, at the end of a unit, merges the two groups'
+//               running max/sum, writes P (bf16 pairs) back into TMEM over
+//               its S row for the PV MMA (A operand from TMEM) and, at the
+//               end of a unit, merges the two groups'
 //               accumulators and stores the output (or a partial).
 // The two softmax groups keep separate O accumulators (TMEM columns), so they
 // never wait on each other inside a unit.
@@ -46,9 +51,10 @@ constexpr int kProducerWarp = 0;
 constexpr int kMmaWarp = 1;
 constexpr int kSoftmaxWarp0 = 2;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemS = 0;      // S of group w at column 64*w
-constexpr uint32_t kTmemO = 128;    // O of group w at column 128 + D*w
-constexpr uint32_t kTmemX = 384;    // (max, sum) exchange between groups
+constexpr int kSBufs = 3;           // S buffers in TMEM (QK runs this far ahead of PV)
+constexpr uint32_t kTmemS = 0;      // S buffer k at column 64*k
+constexpr uint32_t kTmemO = 192;    // O of group w at column 192 + D*w
+constexpr uint32_t kTmemX = 448;    // (max, sum) exchange between groups, 2 columns a slot
 constexpr float kRescaleLog2 = 8.0f;  // rescale O only when the max grows by > 2^8
 
 struct AttnArgs {
@@ -199,26 +205,27 @@ __device__ __forceinline__ bool cursor_next(const AttnArgs& a, SegCursor& c, Seg
 
 template <int D>
 struct AttnLayout {
-  static constexpr int DH = D / 64;                   // 64-column panels per row
-  static constexpr int kStages = (D == 128) ? 5 : 8;  // K/V ring depth
-  static constexpr int kQPanel = kTileM * 128;        // bytes of one Q panel
+  static constexpr int DH = D / 64;                 // 64-column panels per row
+  static constexpr int kNK = (D == 128) ? 5 : 10;   // K ring depth
+  static constexpr int kNV = (D == 128) ? 7 : 14;   // V ring depth
+  static constexpr int kQPanel = kTileM * 128;      // bytes of one Q panel
   static constexpr int kQBytes = DH * kQPanel;
-  static constexpr int kPBytes = kTileM * kTileN * 2;  // one group's P tile
   static constexpr int kKVPanel = kTileN * 128;        // bytes of one K (or V) panel
   static constexpr int kKVBytes = DH * kKVPanel;       // one K (or V) tile
   static constexpr int kQOff = 0;
-  static constexpr int kPOff = kQOff + kQBytes;
-  static constexpr int kKOff = kPOff + 2 * kPBytes;
-  static constexpr int kVOff = kKOff + kStages * kKVBytes;
-  static constexpr int kBarOff = kVOff + kStages * kKVBytes;
+  static constexpr int kKOff = kQOff + kQBytes;
+  static constexpr int kVOff = kKOff + kNK * kKVBytes;
+  static constexpr int kBarOff = kVOff + kNV * kKVBytes;
   // barrier indices
-  static constexpr int kBarKvFull = 0;
-  static constexpr int kBarKvEmpty = kStages;
-  static constexpr int kBarQFull = 2 * kStages;
+  static constexpr int kBarKFull = 0;
+  static constexpr int kBarKEmpty = kBarKFull + kNK;
+  static constexpr int kBarVFull = kBarKEmpty + kNK;
+  static constexpr int kBarVEmpty = kBarVFull + kNV;
+  static constexpr int kBarQFull = kBarVEmpty + kNV;
   static constexpr int kBarQEmpty = kBarQFull + 1;
-  static constexpr int kBarSFull = kBarQEmpty + 1;    // [2]
-  static constexpr int kBarPReady = kBarSFull + 2;    // [2]
-  static constexpr int kBarOReady = kBarPReady + 2;   // [2]
+  static constexpr int kBarSFull = kBarQEmpty + 1;      // [kSBufs]
+  static constexpr int kBarPReady = kBarSFull + kSBufs;  // [2]
+  static constexpr int kBarOReady = kBarPReady + 2;      // [2]
   static constexpr int kBarOFree = kBarOReady + 2;
   static constexpr int kBarXchg = kBarOFree + 1;
   static constexpr int kBarDrain = kBarXchg + 1;
@@ -227,12 +234,14 @@ struct AttnLayout {
   static constexpr int kBytes = kMiscOff + 16;
   static constexpr int kAlloc = kBytes + 1024;  // slack to align the base
   static_assert(kAlloc <= 232448, "shared memory budget exceeded");
+  // QK runs kSBufs tiles ahead of PV: the K ring must hold that many tiles.
+  static_assert(kNK >= kSBufs, "K ring shallower than the QK lead");
 };
 
 // Descriptors of the four MMA operands (all SWIZZLE_128B).
 // A = Q (K-major): panel p at +p*kQPanel, 8-row groups 1024 B apart.
 // B = K tile (K-major): panel p at +p*kKVPanel.
-// A = P (K-major): one 64-key panel.
+// A = P: in TMEM (packed bf16 pairs aliasing the first 32 columns of its S buffer).
 // B = V tile (MN-major): D-panels kKVPanel apart (LBO), 8-key groups 1024 B apart (SBO).
 template <int D>
 __device__ __forceinline__ uint64_t desc_q(uint32_t q, int kk) {
@@ -241,9 +250,6 @@ __device__ __forceinline__ uint64_t desc_q(uint32_t q, int kk) {
 template <int D>
 __device__ __forceinline__ uint64_t desc_k(uint32_t k, int kk) {
   return smem_desc_sw128(k + (kk >> 2) * AttnLayout<D>::kKVPanel + (kk & 3) * 32, 16, 1024);
-}
-__device__ __forceinline__ uint64_t desc_p(uint32_t p, int kk) {
-  return smem_desc_sw128(p + kk * 32, 16, 1024);
 }
 template <int D>
 __device__ __forceinline__ uint64_t desc_v(uint32_t v, int kk) {
@@ -265,6 +271,11 @@ __device__ __forceinline__ void raise_flag(const AttnArgs& a, int bits) {
 // ---------------------------------------------------------------------------
 // Roles
 
+// One thread issues everything: the Q tile of each unit, then per key tile its
+// K copy into the K ring and its V copy into the V ring (one 3-D box each: 64
+// tokens x both 64-column halves of D, landing as the two swizzled panels the
+// MMA descriptors expect). The next page id is read while the current tile's
+// copies are issued.
 template <int D>
 __device__ __forceinline__ void producer_role(const AttnArgs& a, uint8_t* smem,
                                               const CUtensorMap* tm_q, const CUtensorMap* tm_kc,
@@ -273,75 +284,91 @@ __device__ __forceinline__ void producer_role(const AttnArgs& a, uint8_t* smem,
   using Lay = AttnLayout<D>;
   const uint32_t base = smem_u32(smem);
   const uint32_t bars = base + Lay::kBarOff;
-  auto bar = [&](int i) { return bars + 8u * i; };
-  int issued[Lay::kStages];
-#pragma unroll
-  for (int s = 0; s < Lay::kStages; ++s) issued[s] = 0;
-  int q_issued = 0;
+  const uint32_t blk_bytes = Lay::DH * a.blk_box_rows * 128;
+  const int tiles_per_page = a.page_size / kTileN;
+  int kt = 0, vt = 0, q_issued = 0;  // K copies, V copies and Q tiles issued
   bool ok = true;
 
   SegCursor cur;
   cursor_init(a, blockIdx.x, cur);
   Segment sg;
-  int it = 0, si = 0;
+  int si = 0;
   while (ok && cursor_next(a, cur, sg)) {
     const int b = sg.b, h = sg.h;
-    const int Kb = seq_block_len(a, b), row0 = seq_row0(a, b);
+    const int row0 = seq_row0(a, b);
     const int L = seq_prefix_len(a, b);
     const int np = (L + kTileN - 1) / kTileN;
-    (void)Kb;
+    const int* ptab = a.page_table + (long long)b * a.max_pages;
     // Q tile of this unit: rows (i, g) for i < max_block, g < G.
-    if (si > 0 && !mbar_wait(bar(Lay::kBarQEmpty), (si - 1) & 1, abort_flag, a.timeout_ns)) {
+    if (si > 0 && !mbar_wait(bars + 8u * Lay::kBarQEmpty, (si - 1) & 1, abort_flag, a.timeout_ns)) {
       ok = false;
       break;
     }
-    mbar_arrive_expect_tx(bar(Lay::kBarQFull), Lay::DH * a.G * a.q_box_rows * 128);
+    mbar_arrive_expect_tx(bars + 8u * Lay::kBarQFull, Lay::DH * a.G * a.q_box_rows * 128);
+#pragma unroll
     for (int p = 0; p < Lay::DH; ++p)
-      tma_load_3d(base + Lay::kQOff + p * Lay::kQPanel, tm_q, bar(Lay::kBarQFull), p * 64,
+      tma_load_3d(base + Lay::kQOff + p * Lay::kQPanel, tm_q, bars + 8u * Lay::kBarQFull, p * 64,
                   h * a.G, row0);
     ++q_issued;
-    for (int t = sg.t0; t < sg.t1; ++t, ++it) {
-      const int stage = it % Lay::kStages;
-      const int round = it / Lay::kStages;
-      if (round > 0 &&
-          !mbar_wait(bar(Lay::kBarKvEmpty + stage), (round - 1) & 1, abort_flag, a.timeout_ns)) {
-        ok = false;
-        break;
-      }
-      const uint32_t fb = bar(Lay::kBarKvFull + stage);
-      const uint32_t kdst = base + Lay::kKOff + stage * Lay::kKVBytes;
-      const uint32_t vdst = base + Lay::kVOff + stage * Lay::kKVBytes;
-      mbar_arrive_expect_tx(fb, t < np ? 2 * Lay::kKVBytes : 2 * Lay::DH * a.blk_box_rows * 128);
-      ++issued[stage];
-      if (t < np) {
-        const int tok = t * kTileN;
-        const int pidx = tok / a.page_size;
-        int page = a.page_table[(long long)b * a.max_pages + pidx];
+    int page_next = (sg.t0 < np) ? ptab[sg.t0 / tiles_per_page] : 0;
+    for (int t = sg.t0; t < sg.t1; ++t) {
+      const int ks = kt % Lay::kNK, kr = kt / Lay::kNK;
+      const int vs = vt % Lay::kNV, vr = vt / Lay::kNV;
+      const bool block = t >= np;
+      int row = row0;
+      if (!block) {
+        int page = page_next;
+        if (t + 1 < np) page_next = ptab[(t + 1) / tiles_per_page];
         if (page < 0 || page >= a.num_pages) {
           raise_flag(a, ORTHRUS_FLAG_BAD_PAGE);
           page = 0;  // keep the pipeline flowing on an in-bounds page
         }
-        const int row = (page * a.Hkv + h) * a.page_size + (tok % a.page_size);
-        for (int p = 0; p < Lay::DH; ++p) {
-          tma_load_2d(kdst + p * Lay::kKVPanel, tm_kc, fb, p * 64, row);
-          tma_load_2d(vdst + p * Lay::kKVPanel, tm_vc, fb, p * 64, row);
-        }
-      } else {
-        for (int p = 0; p < Lay::DH; ++p) {
-          tma_load_3d(kdst + p * Lay::kKVPanel, tm_kb, fb, p * 64, h, row0);
-          tma_load_3d(vdst + p * Lay::kKVPanel, tm_vb, fb, p * 64, h, row0);
-        }
+        row = (page * a.Hkv + h) * a.page_size + (t % tiles_per_page) * kTileN;
       }
+      const uint32_t bytes = block ? blk_bytes : (uint32_t)Lay::kKVBytes;
+      // K into its ring (freed by the tile's QK), V into the deeper V ring (freed by PV)
+      if (kr > 0 && !mbar_wait(bars + 8u * (Lay::kBarKEmpty + ks), (kr - 1) & 1, abort_flag,
+                               a.timeout_ns)) { ok = false; break; }
+      const uint32_t kfb = bars + 8u * (Lay::kBarKFull + ks);
+      const uint32_t kdst = base + Lay::kKOff + ks * Lay::kKVBytes;
+      mbar_arrive_expect_tx(kfb, bytes);
+      if (block) {
+#pragma unroll
+        for (int p = 0; p < Lay::DH; ++p)
+          tma_load_3d(kdst + p * Lay::kKVPanel, tm_kb, kfb, p * 64, h, row);
+      } else {
+        tma_load_3d(kdst, tm_kc, kfb, 0, row, 0);
+      }
+      ++kt;
+      if (vr > 0 && !mbar_wait(bars + 8u * (Lay::kBarVEmpty + vs), (vr - 1) & 1, abort_flag,
+                               a.timeout_ns)) { ok = false; break; }
+      const uint32_t vfb = bars + 8u * (Lay::kBarVFull + vs);
+      const uint32_t vdst = base + Lay::kVOff + vs * Lay::kKVBytes;
+      mbar_arrive_expect_tx(vfb, bytes);
+      if (block) {
+#pragma unroll
+        for (int p = 0; p < Lay::DH; ++p)
+          tma_load_3d(vdst + p * Lay::kKVPanel, tm_vb, vfb, p * 64, h, row);
+      } else {
+        tma_load_3d(vdst, tm_vc, vfb, 0, row, 0);
+      }
+      ++vt;
     }
     ++si;
   }
   if (!ok || *abort_flag) {
     // Wind down: let every copy this thread started land before the CTA exits.
     volatile int no_abort = 0;
-    for (int s = 0; s < Lay::kStages; ++s)
-      if (issued[s] > 0)
-        mbar_wait(bar(Lay::kBarKvFull + s), (issued[s] - 1) & 1, &no_abort, 20000000ull);
-    if (q_issued > 0) mbar_wait(bar(Lay::kBarQFull), (q_issued - 1) & 1, &no_abort, 20000000ull);
+    for (int s = 0; s < Lay::kNK; ++s) {
+      const int n = kt / Lay::kNK + (s < kt % Lay::kNK ? 1 : 0);
+      if (n > 0) mbar_wait(bars + 8u * (Lay::kBarKFull + s), (n - 1) & 1, &no_abort, 20000000ull);
+    }
+    for (int s = 0; s < Lay::kNV; ++s) {
+      const int n = vt / Lay::kNV + (s < vt % Lay::kNV ? 1 : 0);
+      if (n > 0) mbar_wait(bars + 8u * (Lay::kBarVFull + s), (n - 1) & 1, &no_abort, 20000000ull);
+    }
+    if (q_issued > 0)
+      mbar_wait(bars + 8u * Lay::kBarQFull, (q_issued - 1) & 1, &no_abort, 20000000ull);
   }
 }
 
@@ -373,6 +400,9 @@ __device__ __forceinline__ bool step_next(const AttnArgs& a, TileStep& s) {
   return true;
 }
 
+// The issuing thread's scalar work sits between consecutive MMAs, so every
+// operand descriptor is a precomputed base plus a compile-time step: the
+// 14-bit start-address field holds (smem address >> 4) and never carries.
 template <int D>
 __device__ __forceinline__ void mma_role(const AttnArgs& a, uint8_t* smem, uint32_t tmem,
                                          volatile int* abort_flag) {
@@ -380,31 +410,39 @@ __device__ __forceinline__ void mma_role(const AttnArgs& a, uint8_t* smem, uint3
   const int lane = threadIdx.x & 31;
   const uint32_t base = smem_u32(smem);
   const uint32_t bars = base + Lay::kBarOff;
-  auto bar = [&](int i) { return bars + 8u * i; };
   constexpr uint32_t kIdescQK = idesc_bf16_f32(kTileM, kTileN, 0);
   constexpr uint32_t kIdescPV = idesc_bf16_f32(kTileM, D, 1);
+  const uint64_t dq = smem_desc_sw128(base + Lay::kQOff, 16, 1024);
+  const uint64_t dk = smem_desc_sw128(base + Lay::kKOff, 16, 1024);
+  const uint64_t dv = smem_desc_sw128(base + Lay::kVOff, Lay::kKVPanel, 1024);
 
-  // Lane 0 waits; the verdict is shared so the warp stays converged.
+  // Every lane polls the barrier (no divergence around the wait); a vote makes
+  // the verdict warp-uniform.
   auto wait = [&](uint32_t b, uint32_t parity) -> bool {
-    int ok = 1;
-    if (lane == 0) ok = mbar_wait(b, parity, abort_flag, a.timeout_ns) ? 1 : 0;
-    return __shfl_sync(0xffffffffu, ok, 0) != 0;
+    const bool ok = mbar_wait(b, parity, abort_flag, a.timeout_ns);
+    return __all_sync(0xffffffffu, ok);
   };
 
+  // S buffer it % 3 is free again once the softmax group has published P for
+  // tile it - 3, which issue_pv of that tile waited for.
   auto issue_qk = [&](const TileStep& j) -> bool {
-    const int stage = j.it % Lay::kStages;
-    if (j.t == j.sg.t0 && !wait(bar(Lay::kBarQFull), j.si & 1)) return false;
-    if (!wait(bar(Lay::kBarKvFull + stage), (j.it / Lay::kStages) & 1)) return false;
+    const int slot = j.it % Lay::kNK;
+    if (!wait(bars + 8u * (Lay::kBarKFull + slot), (j.it / Lay::kNK) & 1)) return false;
+    if (j.t == j.sg.t0 && !wait(bars + 8u * Lay::kBarQFull, j.si & 1)) return false;
     tc_fence_after();
-    if (lane == 0) {
-      const uint32_t q = base + Lay::kQOff;
-      const uint32_t k = base + Lay::kKOff + stage * Lay::kKVBytes;
-      const uint32_t d = tmem + kTmemS + 64u * (j.it & 1);
+    const int sb = j.it % kSBufs;
+    const uint32_t d = tmem + kTmemS + 64u * sb;
+    const uint64_t kd = dk + (uint64_t)((slot * Lay::kKVBytes) >> 4);
 #pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk)
-        mma_bf16_ss(d, desc_q<D>(q, kk), desc_k<D>(k, kk), kIdescQK, kk > 0 ? 1u : 0u);
-      mma_commit(bar(Lay::kBarSFull + (j.it & 1)));
-      if (j.t == j.sg.t1 - 1) mma_commit(bar(Lay::kBarQEmpty));
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const uint64_t aq = dq + (uint64_t)(((kk >> 2) * Lay::kQPanel + (kk & 3) * 32) >> 4);
+      const uint64_t bk = kd + (uint64_t)(((kk >> 2) * Lay::kKVPanel + (kk & 3) * 32) >> 4);
+      if (elect_one()) mma_bf16_ss(d, aq, bk, kIdescQK, kk > 0 ? 1u : 0u);
+    }
+    if (elect_one()) {
+      mma_commit(bars + 8u * (Lay::kBarSFull + sb));
+      mma_commit(bars + 8u * (Lay::kBarKEmpty + slot));
+      if (j.t == j.sg.t1 - 1) mma_commit(bars + 8u * Lay::kBarQEmpty);
     }
     __syncwarp();
     return true;
@@ -412,14 +450,16 @@ __device__ __forceinline__ void mma_role(const AttnArgs& a, uint8_t* smem, uint3
 
   auto issue_pv = [&](const TileStep& j) -> bool {
     const int w = j.it & 1;
-    const int stage = j.it % Lay::kStages;
-    if (!wait(bar(Lay::kBarPReady + w), (j.it >> 1) & 1)) return false;
-    if (j.t == j.sg.t0 && j.si > 0 && !wait(bar(Lay::kBarOFree), (j.si - 1) & 1)) return false;
+    const int slot = j.it % Lay::kNV;
+    // p_ready also means the tile's V copy has landed: the softmax group waits
+    // for it before publishing P, which keeps that wait off this warp's path.
+    if (!wait(bars + 8u * (Lay::kBarPReady + w), (j.it >> 1) & 1)) return false;
+    if (j.t == j.sg.t0 && j.si > 0 && !wait(bars + 8u * Lay::kBarOFree, (j.si - 1) & 1)) return false;
     const int nvalid = tile_valid_keys(j.t, j.L, j.np, j.Kb);
-    const uint32_t v = base + Lay::kVOff + stage * Lay::kKVBytes;
     if (nvalid < kTileN) {
       // Rows past the last valid key may hold stale or non-finite data;
       // P is zero there, but 0 * NaN is NaN, so clear those V rows.
+      const uint32_t v = base + Lay::kVOff + slot * Lay::kKVBytes;
       const int rows = kTileN - nvalid;
       const int chunks = rows * Lay::DH * 8;  // 16-byte chunks
       for (int c = lane; c < chunks; c += 32) {
@@ -432,15 +472,21 @@ __device__ __forceinline__ void mma_role(const AttnArgs& a, uint8_t* smem, uint3
       __syncwarp();
     }
     tc_fence_after();
-    if (lane == 0) {
-      const uint32_t pbuf = base + Lay::kPOff + w * Lay::kPBytes;
-      const uint32_t d = tmem + kTmemO + (uint32_t)(D * w);
-      const uint32_t acc0 = (j.t - j.sg.t0 >= 2) ? 1u : 0u;
+    // P of this tile sits in the first 32 columns of its S buffer; the next QK
+    // into that buffer is issued after this PV, and the tensor pipe runs one
+    // thread's MMAs in order, so P is read before it is overwritten.
+    const uint32_t pa = tmem + kTmemS + 64u * (j.it % kSBufs);
+    const uint64_t vd = dv + (uint64_t)((slot * Lay::kKVBytes) >> 4);
+    const uint32_t d = tmem + kTmemO + (uint32_t)(D * w);
+    const uint32_t acc0 = (j.t - j.sg.t0 >= 2) ? 1u : 0u;
 #pragma unroll
-      for (int kk = 0; kk < kTileN / 16; ++kk)
-        mma_bf16_ss(d, desc_p(pbuf, kk), desc_v<D>(v, kk), kIdescPV, (kk > 0) ? 1u : acc0);
-      mma_commit(bar(Lay::kBarOReady + w));
-      mma_commit(bar(Lay::kBarKvEmpty + stage));
+    for (int kk = 0; kk < kTileN / 16; ++kk) {
+      const uint64_t bv = vd + (uint64_t)((kk * 16 * 128) >> 4);
+      if (elect_one()) mma_bf16_ts(d, pa + 8u * kk, bv, kIdescPV, (kk > 0) ? 1u : acc0);
+    }
+    if (elect_one()) {
+      mma_commit(bars + 8u * (Lay::kBarOReady + w));
+      mma_commit(bars + 8u * (Lay::kBarVEmpty + slot));
     }
     __syncwarp();
     return true;
@@ -453,19 +499,17 @@ __device__ __forceinline__ void mma_role(const AttnArgs& a, uint8_t* smem, uint3
   qs.valid = false;
   ps = qs;
   bool ok = true;
-  if (step_next(a, qs)) ok = issue_qk(qs);
+  for (int k = 0; k < kSBufs && ok; ++k)
+    if (step_next(a, qs)) ok = issue_qk(qs);
   while (ok && step_next(a, ps)) {
-    const bool have_next = step_next(a, qs);
-    const bool same_seg = have_next && qs.si == ps.si;
-    if (same_seg) ok = issue_qk(qs);
-    if (ok) ok = issue_pv(ps);
-    if (ok && have_next && !same_seg) ok = issue_qk(qs);
+    ok = issue_pv(ps);
+    if (ok && step_next(a, qs)) ok = issue_qk(qs);
   }
   // Drain: every MMA issued above completes before TMEM is released.
   if (lane == 0) {
-    mma_commit(bar(Lay::kBarDrain));
+    mma_commit(bars + 8u * Lay::kBarDrain);
     volatile int no_abort = 0;
-    mbar_wait(bar(Lay::kBarDrain), 0, &no_abort, 20000000ull);
+    mbar_wait(bars + 8u * Lay::kBarDrain, 0, &no_abort, 20000000ull);
   }
   __syncwarp();
 }
@@ -482,11 +526,9 @@ __device__ __forceinline__ void softmax_role(const AttnArgs& a, uint8_t* smem, u
   const uint32_t base = smem_u32(smem);
   const uint32_t bars = base + Lay::kBarOff;
   auto bar = [&](int i) { return bars + 8u * i; };
-  const uint32_t t_s = tmem + lane_off + kTmemS + 64u * w;
   const uint32_t t_o_self = tmem + lane_off + kTmemO + (uint32_t)(D * w);
   const uint32_t t_o0 = tmem + lane_off + kTmemO;
   const uint32_t t_o1 = tmem + lane_off + kTmemO + D;
-  const uint32_t pbuf = base + Lay::kPOff + w * Lay::kPBytes;
   const float c = a.scale_log2;
   const float NEG_INF = -__int_as_float(0x7f800000);
 
@@ -519,9 +561,11 @@ __device__ __forceinline__ void softmax_role(const AttnArgs& a, uint8_t* smem, u
 
     for (int t = sg.t0; t < sg.t1; ++t, ++it) {
       if ((it & 1) != w) continue;
-      if (!wait(bar(Lay::kBarSFull + w), (it >> 1) & 1)) { ok = false; break; }
+      const int sb = it % kSBufs;
+      if (!wait(bar(Lay::kBarSFull + sb), (it / kSBufs) & 1)) { ok = false; break; }
       tc_fence_after();
       float s[64];
+      const uint32_t t_s = tmem + lane_off + kTmemS + 64u * sb;
       tmem_ld32(t_s, *reinterpret_cast<float(*)[32]>(&s[0]));
       tmem_ld32(t_s + 32, *reinterpret_cast<float(*)[32]>(&s[32]));
       tmem_wait_ld();
@@ -534,14 +578,18 @@ __device__ __forceinline__ void softmax_role(const AttnArgs& a, uint8_t* smem, u
 #pragma unroll
         for (int k = 0; k < 64; ++k) s[k] = (k < lim) ? s[k] : NEG_INF;
       }
-      float mt = NEG_INF;
+      float mx[8];
 #pragma unroll
-      for (int k = 0; k < 64; ++k) mt = fmaxf(mt, s[k]);
+      for (int k = 0; k < 8; ++k) mx[k] = s[k];
+#pragma unroll
+      for (int k = 8; k < 64; ++k) mx[k & 7] = fmaxf(mx[k & 7], s[k]);
+      const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                             fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
       const float m_new = fmaxf(m_ref, mt * c);
       const bool need = has && (m_new > m_ref + kRescaleLog2);
       if (!has) m_ref = m_new;
-      // The previous PV of this group must be done before P is overwritten
-      // (and before O is rescaled).
+      // The previous PV of this group must be done before O is rescaled (and
+      // the wait keeps this group's o_ready phases in step).
       if (cnt > 0 && pv_waited < cnt) {
         if (!wait(bar(Lay::kBarOReady + w), pv_waited & 1)) { ok = false; break; }
         ++pv_waited;
@@ -565,22 +613,27 @@ __device__ __forceinline__ void softmax_role(const AttnArgs& a, uint8_t* smem, u
         tmem_wait_st();
       }
       const float mref = (m_ref == NEG_INF) ? 0.f : m_ref;
-      float rsum = 0.f;
+      float psum[8];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        float p[8];
+      for (int k = 0; k < 8; ++k) psum[k] = 0.f;
+      uint32_t pk[32];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          p[k] = ex2_approx(fmaf(s[8 * q + k], c, -mref));
-          rsum += p[k];
-        }
-        const uint32_t addr = pbuf + row * 128 + ((q ^ (row & 7)) << 4);
-        st_shared_v4(addr, pack_bf16x2(p[0], p[1]), pack_bf16x2(p[2], p[3]),
-                     pack_bf16x2(p[4], p[5]), pack_bf16x2(p[6], p[7]));
+      for (int k = 0; k < 32; ++k) {
+        const float p0 = ex2_approx(fmaf(s[2 * k], c, -mref));
+        const float p1 = ex2_approx(fmaf(s[2 * k + 1], c, -mref));
+        psum[(2 * k) & 7] += p0;
+        psum[(2 * k + 1) & 7] += p1;
+        pk[k] = pack_bf16x2(p0, p1);
       }
-      l_sum += rsum;
+      // P (bf16 pairs) over the first 32 columns of this tile's S buffer
+      tmem_st32u(t_s, pk);
+      if (!wait(bars + 8u * (Lay::kBarVFull + it % Lay::kNV), (it / Lay::kNV) & 1)) {
+        ok = false;
+        break;
+      }
+      l_sum += ((psum[0] + psum[1]) + (psum[2] + psum[3])) + ((psum[4] + psum[5]) + (psum[6] + psum[7]));
       has = true;
-      fence_proxy_async_smem();
+      tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(Lay::kBarPReady + w));
       ++cnt;
@@ -592,28 +645,15 @@ __device__ __forceinline__ void softmax_role(const AttnArgs& a, uint8_t* smem, u
       if (!wait(bar(Lay::kBarOReady + w), pv_waited & 1)) { ok = false; break; }
       ++pv_waited;
     }
-    {
-      float x[32];
-      x[0] = m_ref;
-      x[1] = l_sum;
-      // only columns 0..1 matter; a 32-column store keeps one code path
-#pragma unroll
-      for (int k = 2; k < 32; ++k) x[k] = 0.f;
-      tmem_st32(tmem + lane_off + kTmemX + 32u * ((si & 1) * 2 + w), x);
-      tmem_wait_st();
-    }
+    tmem_st2(tmem + lane_off + kTmemX + 2u * ((si & 1) * 2 + w), m_ref, l_sum);
+    tmem_wait_st();
     tc_fence_before();
     mbar_arrive(bar(Lay::kBarXchg));
     if (!wait(bar(Lay::kBarXchg), si & 1)) { ok = false; break; }
     tc_fence_after();
     float m_o, l_o;
-    {
-      float x[32];
-      tmem_ld32(tmem + lane_off + kTmemX + 32u * ((si & 1) * 2 + (1 - w)), x);
-      tmem_wait_ld();
-      m_o = x[0];
-      l_o = x[1];
-    }
+    tmem_ld2(tmem + lane_off + kTmemX + 2u * ((si & 1) * 2 + (1 - w)), m_o, l_o);
+    tmem_wait_ld();
     const float m0 = w == 0 ? m_ref : m_o, l0 = w == 0 ? l_sum : l_o;
     const float m1 = w == 0 ? m_o : m_ref, l1 = w == 0 ? l_o : l_sum;
     float M = NEG_INF;
@@ -667,7 +707,6 @@ __device__ __forceinline__ void softmax_role(const AttnArgs& a, uint8_t* smem, u
       a.ws_lse[(long long)sg.part * kTileM + row] = M + log2f(Lt);
     tc_fence_before();
     mbar_arrive(bar(Lay::kBarOFree));
-    (void)b;
     ++si;
   }
 }
@@ -687,6 +726,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::kMiscOff + 4);
   const int warp = threadIdx.x >> 5;
 
+  // The combine kernel may be scheduled as soon as every CTA got here; it
+  // waits for this grid's writes before it reads them.
+  pdl_launch_dependents();
+
   // A CTA whose range is empty has nothing to set up.
   {
     SegCursor cur;
@@ -696,14 +739,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   if (threadIdx.x == 0) {
     const uint32_t bars = smem_u32(smem) + Lay::kBarOff;
-    for (int s = 0; s < Lay::kStages; ++s) {
-      mbar_init(bars + 8u * (Lay::kBarKvFull + s), 1);
-      mbar_init(bars + 8u * (Lay::kBarKvEmpty + s), 1);
+    for (int s = 0; s < Lay::kNK; ++s) {
+      mbar_init(bars + 8u * (Lay::kBarKFull + s), 1);
+      mbar_init(bars + 8u * (Lay::kBarKEmpty + s), 1);
+    }
+    for (int s = 0; s < Lay::kNV; ++s) {
+      mbar_init(bars + 8u * (Lay::kBarVFull + s), 1);
+      mbar_init(bars + 8u * (Lay::kBarVEmpty + s), 1);
     }
     mbar_init(bars + 8u * Lay::kBarQFull, 1);
     mbar_init(bars + 8u * Lay::kBarQEmpty, 1);
+    for (int k = 0; k < kSBufs; ++k) mbar_init(bars + 8u * (Lay::kBarSFull + k), 1);
     for (int w = 0; w < 2; ++w) {
-      mbar_init(bars + 8u * (Lay::kBarSFull + w), 1);
       mbar_init(bars + 8u * (Lay::kBarPReady + w), 128);
       mbar_init(bars + 8u * (Lay::kBarOReady + w), 1);
     }
@@ -747,7 +794,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
 // ---------------------------------------------------------------------------
 // Combine: merge the partials of every unit that was cut across CTAs.
-// grid = (B * Hkv, 128 / kCombineRows); 32 threads per query row.
+// grid = (B * Hkv, ceil(G * max_block / kCombineRows)); one warp per query row.
+// Warp 0 finds the unit's partials once per CTA; the partials themselves are
+// read only after the attention grid's writes are visible (griddepcontrol.wait).
 
 constexpr int kCombineRows = 8;
 
@@ -762,48 +811,74 @@ __device__ __forceinline__ int cta_of_tile(long long T, int C, long long t) {
 template <int D>
 __global__ void __launch_bounds__(kCombineRows * 32)
     attn_combine_kernel(const AttnArgs a) {
+  __shared__ long long sh_T, sh_su;
+  __shared__ int sh_clo, sh_chi, sh_count, sh_skip;
   const int u = blockIdx.x;
   const int b = u / a.Hkv, h = u % a.Hkv;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (u == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
     for (int bb = 0; bb < a.B; ++bb)
       if (seq_rows_bad(a, bb) || seq_len_bad(a, bb)) raise_flag(a, ORTHRUS_FLAG_BAD_LENGTH);
   }
-  const int Kb = seq_block_len(a, b);
-  if (b >= a.B || Kb <= 0) return;
+  const int Kb = (b < a.B) ? seq_block_len(a, b) : 0;
+  if (Kb <= 0) return;
   const int nt = seq_tiles(a, b);
-  const int r = blockIdx.y * kCombineRows + (threadIdx.x >> 5);
+  if (warp == 0) {
+    int skip = 0, count = 0, c_lo = 0, c_hi = -1;
+    long long T = 0, s_u = 0;
+    if (a.chunked) {
+      count = unit_chunks(a, nt);
+      skip = count <= 1;
+    } else {
+      // total tiles and this unit's first tile, summed across the warp
+      long long t_part = 0, s_part = 0;
+      for (int bb = lane; bb < a.B; bb += 32) {
+        const long long n = (long long)a.Hkv * seq_tiles(a, bb);
+        t_part += n;
+        if (bb < b) s_part += n;
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        t_part += __shfl_xor_sync(0xffffffffu, t_part, o);
+        s_part += __shfl_xor_sync(0xffffffffu, s_part, o);
+      }
+      T = t_part;
+      s_u = s_part + (long long)h * nt;
+      c_lo = cta_of_tile(T, a.num_ctas, s_u);
+      c_hi = cta_of_tile(T, a.num_ctas, s_u + nt - 1);
+      skip = c_lo == c_hi;
+      count = c_hi - c_lo + 1;
+    }
+    if (lane == 0) {
+      sh_T = T;
+      sh_su = s_u;
+      sh_clo = c_lo;
+      sh_chi = c_hi;
+      sh_count = count;
+      sh_skip = skip;
+    }
+  }
+  __syncthreads();
+  if (sh_skip) return;
+  const int r = blockIdx.y * kCombineRows + warp;
   if (r >= a.G * Kb) return;
-  const int lane = threadIdx.x & 31;
+  const long long T = sh_T, s_u = sh_su;
+  const int c_lo = sh_clo, count = sh_count;
   constexpr int kPer = D / 32;  // elements per thread
 
-  // Partials of this unit: parts p_lo.. in chunked mode, the CTAs of the
-  // covering range (empty CTAs skipped) in balanced mode.
-  int n_parts = 0;
-  int c_lo = 0, c_hi = -1;
-  long long T = 0, s_u = 0;
-  if (a.chunked) {
-    n_parts = unit_chunks(a, nt);
-    if (n_parts <= 1) return;
-  } else {
-    T = total_tiles(a);
-    for (int bb = 0; bb < b; ++bb) s_u += (long long)a.Hkv * seq_tiles(a, bb);
-    s_u += (long long)h * nt;
-    c_lo = cta_of_tile(T, a.num_ctas, s_u);
-    c_hi = cta_of_tile(T, a.num_ctas, s_u + nt - 1);
-    if (c_lo == c_hi) return;
-  }
   auto part_of = [&](int k, bool& use) -> int {
     if (a.chunked) {
       use = true;
       return u * a.max_chunks + k;
     }
     const int cc = c_lo + k;
-    use = range_begin(T, cc, a.num_ctas) < range_begin(T, cc + 1, a.num_ctas);
-    const int slot = (cc == c_lo && s_u > range_begin(T, cc, a.num_ctas)) ? 1 : 0;
+    const long long beg = range_begin(T, cc, a.num_ctas);
+    use = beg < range_begin(T, cc + 1, a.num_ctas);
+    const int slot = (cc == c_lo && s_u > beg) ? 1 : 0;
     return cc * 2 + slot;
   };
-  const int count = a.chunked ? n_parts : (c_hi - c_lo + 1);
 
+  pdl_wait();  // partials written by the attention grid are visible from here on
   float M = -__int_as_float(0x7f800000);
   for (int k = 0; k < count; ++k) {
     bool use;

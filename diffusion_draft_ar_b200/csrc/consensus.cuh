@@ -16,6 +16,8 @@
 
 #include <cstdint>
 
+#include "ptx.cuh"
+
 namespace orthrus {
 
 constexpr int kConsThreads = 256;
@@ -65,6 +67,7 @@ __global__ void __launch_bounds__(kConsThreads)
     consensus_argmax_kernel(const float* __restrict__ logits, long long ld, int V,
                             const int* __restrict__ cu_block, int B, int max_block, int n_chunks,
                             unsigned long long* __restrict__ part) {
+  pdl_launch_dependents();  // the finalize pass may start its launch now
   const int r = blockIdx.y;
   const int R = cu_block ? cu_block[B] : B * max_block;
   if (r >= R) return;
@@ -148,6 +151,7 @@ __global__ void consensus_finalize_kernel(const unsigned long long* __restrict__
     }
     return;
   }
+  pdl_wait();  // the argmax pass's keys are visible from here on
   int m = Kb;  // leading matches
   int next = -1;
   for (int base = 0; base < Kb; base += 32) {

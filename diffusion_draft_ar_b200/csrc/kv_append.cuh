@@ -5,7 +5,10 @@
 //
 // One CTA per sequence copies its accepted rows' K and V (VERIFY view) into the
 // slots L_b .. L_b + n_b - 1 of its pages with 16-byte loads and stores, then
-// (optionally) advances prefix_lens[b] once every row found its page.
+// (optionally) advances prefix_lens[b] once every row found its page. The ids of
+// the first kMaxAppendPages pages the rows land in are read once into shared
+// memory (rows rarely span more than two pages), so the copies carry no
+// dependent loads. A row whose page is out of range is skipped and flagged.
 #pragma once
 
 #include <cstdint>
@@ -14,7 +17,8 @@
 
 namespace orthrus {
 
-constexpr int kAppendThreads = 256;
+constexpr int kAppendThreads = 512;
+constexpr int kMaxAppendPages = 8;
 
 __global__ void __launch_bounds__(kAppendThreads)
     kv_append_kernel(const uint4* __restrict__ k_block, const uint4* __restrict__ v_block,
@@ -23,51 +27,84 @@ __global__ void __launch_bounds__(kAppendThreads)
                      const int* __restrict__ page_table, int max_pages, int num_pages,
                      uint4* k_cache, uint4* v_cache, int Hkv, int D, int page_size,
                      int* error_flag) {
+  __shared__ int sh_page[kMaxAppendPages];
+  __shared__ int sh_flags;
   const int b = blockIdx.x;
   const int row0 = cu_block ? cu_block[b] : b * max_block;
   const int Kb = cu_block ? cu_block[b + 1] - row0 : max_block;
   const int L = prefix_lens[b];
   const int n = accept_len[b];
   const int cpr = D / 8;  // 16-byte chunks per head row
-  int flags = 0;
-  if (n < 0 || n > Kb || L < 0) flags |= ORTHRUS_FLAG_BAD_LENGTH;
-  if (!flags) {
+  const bool seq_bad = n < 0 || n > Kb || L < 0;
+  const long long p_first = seq_bad ? 0 : L / page_size;
+
+  // page id of page index pidx, or -1 (and a flag) when it is out of range
+  auto page_of = [&](long long pidx) -> int {
+    if (pidx >= max_pages) {
+      atomicOr(&sh_flags, ORTHRUS_FLAG_BAD_LENGTH);
+      return -1;
+    }
+    const int page = page_table[static_cast<long long>(b) * max_pages + pidx];
+    if (page < 0 || page >= num_pages) {
+      atomicOr(&sh_flags, ORTHRUS_FLAG_BAD_PAGE);
+      return -1;
+    }
+    return page;
+  };
+
+  if (threadIdx.x == 0) sh_flags = 0;
+  __syncthreads();
+  if (!seq_bad && n > 0) {
+    const long long n_pages = (static_cast<long long>(L) + n - 1) / page_size - p_first + 1;
+    if (threadIdx.x < kMaxAppendPages && threadIdx.x < n_pages)
+      sh_page[threadIdx.x] = page_of(p_first + threadIdx.x);
+  }
+  // every thread has read L (and the page ids are in place) from here on
+  __syncthreads();
+  if (!seq_bad) {
     const int items = n * Hkv * cpr;
-    for (int it = threadIdx.x; it < items; it += blockDim.x) {
-      const int c = it % cpr;
-      const int rest = it / cpr;
-      const int h = rest % Hkv;
-      const int i = rest / Hkv;
-      const long long pos = static_cast<long long>(L) + i;
-      const long long pidx = pos / page_size;
-      if (pidx >= max_pages) {
-        flags |= ORTHRUS_FLAG_BAD_LENGTH;
-        continue;
+    constexpr int U = 4;
+    for (int base = threadIdx.x; base < items; base += U * kAppendThreads) {
+      uint4 kv[U], vv[U];
+      long long dst[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int it = base + u * kAppendThreads;
+        dst[u] = -1;
+        if (it < items) {
+          const int c = it % cpr;
+          const int rest = it / cpr;
+          const int h = rest % Hkv;
+          const int i = rest / Hkv;
+          const long long pos = static_cast<long long>(L) + i;
+          const long long k = pos / page_size - p_first;
+          const int page = k < kMaxAppendPages ? sh_page[k] : page_of(pos / page_size);
+          if (page >= 0) {
+            const long long slot = pos % page_size;
+            dst[u] = ((static_cast<long long>(page) * Hkv + h) * page_size + slot) * cpr + c;
+            const long long src = (static_cast<long long>(row0 + i) * Hkv + h) * cpr + c;
+            kv[u] = k_block[src];
+            vv[u] = v_block[src];
+          }
+        }
       }
-      const int page = page_table[static_cast<long long>(b) * max_pages + pidx];
-      if (page < 0 || page >= num_pages) {
-        flags |= ORTHRUS_FLAG_BAD_PAGE;
-        continue;
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        if (dst[u] >= 0) {
+          k_cache[dst[u]] = kv[u];
+          v_cache[dst[u]] = vv[u];
+        }
       }
-      const long long slot = pos % page_size;
-      const long long dst = ((static_cast<long long>(page) * Hkv + h) * page_size + slot) * cpr + c;
-      const long long src = (static_cast<long long>(row0 + i) * Hkv + h) * cpr + c;
-      k_cache[dst] = k_block[src];
-      v_cache[dst] = v_block[src];
     }
   }
-  // every thread has read L before anyone may change it
-  const int any = __syncthreads_or(flags);
-  if (any) {
-    // collect the flag bits of the whole block
-    __shared__ int bits;
-    if (threadIdx.x == 0) bits = 0;
-    __syncthreads();
-    if (flags) atomicOr(&bits, flags);
-    __syncthreads();
-    if (threadIdx.x == 0 && error_flag) atomicOr(error_flag, bits);
-  } else if (update_lens && threadIdx.x == 0) {
-    prefix_lens[b] = L + n;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const int flags = seq_bad ? ORTHRUS_FLAG_BAD_LENGTH : sh_flags;
+    if (flags) {
+      if (error_flag) atomicOr(error_flag, flags);
+    } else if (update_lens) {
+      prefix_lens[b] = L + n;
+    }
   }
 }
 

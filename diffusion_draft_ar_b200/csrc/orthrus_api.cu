@@ -191,12 +191,14 @@ orthrus_status_t launch_attn(const orthrus_attn_params* p, const AttnPlan& pl, i
       return fail(ORTHRUS_ERR_CUDA, "tensor map for q_block");
   }
   {
+    // cache rows (one token of one head) viewed as (64 columns, row, D/64 halves):
+    // one box of {64, 64, D/64} lands as D/64 panels of 64 rows x 128 bytes
     const cuuint64_t rows = (cuuint64_t)p->num_pages * p->Hkv * p->page_size;
-    const cuuint64_t dims[2] = {(cuuint64_t)D, rows > 0 ? rows : 1};
-    const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
-    const cuuint32_t box[2] = {64, (cuuint32_t)kTileN};
-    if (!make_map(&tkc, p->k_cache, 2, dims, strides, box) ||
-        !make_map(&tvc, p->v_cache, 2, dims, strides, box))
+    const cuuint64_t dims[3] = {64, rows > 0 ? rows : 1, (cuuint64_t)D / 64};
+    const cuuint64_t strides[2] = {(cuuint64_t)D * 2, 128};
+    const cuuint32_t box[3] = {64, (cuuint32_t)kTileN, (cuuint32_t)D / 64};
+    if (!make_map(&tkc, p->k_cache, 3, dims, strides, box) ||
+        !make_map(&tvc, p->v_cache, 3, dims, strides, box))
       return fail(ORTHRUS_ERR_CUDA, "tensor map for the KV cache");
   }
   {
@@ -238,10 +240,21 @@ orthrus_status_t launch_attn(const orthrus_attn_params* p, const AttnPlan& pl, i
   block_attn_kernel<D><<<pl.grid, kAttnThreads, Lay::kAlloc, stream>>>(tq, tkc, tvc, tkb, tvb, a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return fail(ORTHRUS_ERR_CUDA, "block_attn launch: %s", cudaGetErrorString(e));
+  // The combine kernel is launched as a programmatic dependent of the
+  // attention grid: its launch and schedule prologue overlap the attention
+  // tail, and it reads the partials only after griddepcontrol.wait.
   const int row_groups = (pl.G * p->max_block + kCombineRows - 1) / kCombineRows;
-  dim3 cgrid(p->B * p->Hkv, row_groups);
-  attn_combine_kernel<D><<<cgrid, kCombineRows * 32, 0, stream>>>(a);
-  e = cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p->B * p->Hkv, row_groups);
+  cfg.blockDim = dim3(kCombineRows * 32);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, attn_combine_kernel<D>, a);
   if (e != cudaSuccess) return fail(ORTHRUS_ERR_CUDA, "combine launch: %s", cudaGetErrorString(e));
   return ok();
 }
@@ -327,10 +340,21 @@ orthrus_status_t orthrus_consensus(const float* verify_logits, int64_t ld, int32
                                                           max_block, n_chunks, part);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return fail(ORTHRUS_ERR_CUDA, "consensus launch: %s", cudaGetErrorString(e));
+  // finalize is a programmatic dependent of the argmax pass: its launch
+  // overlaps the argmax tail and it reads the keys after griddepcontrol.wait
   const int warps = 8;
-  consensus_finalize_kernel<<<(B + warps - 1) / warps, warps * 32, 0, st>>>(
-      part, n_chunks, draft_tokens, cu_block, B, max_block, accept_len, next_token, row_argmax);
-  e = cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((B + warps - 1) / warps);
+  cfg.blockDim = dim3(warps * 32);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, consensus_finalize_kernel, static_cast<const unsigned long long*>(part),
+                         n_chunks, draft_tokens, cu_block, static_cast<int>(B),
+                         static_cast<int>(max_block), accept_len, next_token, row_argmax);
   if (e != cudaSuccess) return fail(ORTHRUS_ERR_CUDA, "consensus launch: %s", cudaGetErrorString(e));
   return ok();
 }
