@@ -16,15 +16,17 @@
 // the prefix lengths; a unit cut by a range boundary is finished by the combine
 // kernel from per-CTA partials (max, sum, normalised accumulator).
 //
-// Roles (320 threads):
+// Roles (352 threads):
 //   warp 0      TMA producer: Q tile per unit; K tiles into a K ring and V
 //               tiles into a separate, deeper V ring (K is released by its
 //               QK three tiles before V is released by its PV); the next
 //               page id is fetched while the current tile's copies are issued.
-//   warp 1      MMA issuer: S = Q K^T into one of three TMEM S buffers, running
-//               three tiles ahead of O += P V, so a softmax group never waits
-//               for a QK round trip; owns TMEM.
-//   warps 2-5   softmax group 0 (even tiles), warps 6-9 softmax group 1 (odd
+//   warps 1-2   MMA issuers, one per softmax group: S = Q K^T for the group's
+//               tiles into its two TMEM S buffers (one own tile ahead), and
+//               O += P V into its TMEM accumulator. Two issuing warps overlap
+//               the per-tile issue overhead; each keeps its own P/S aliasing
+//               in one in-order MMA stream. Warp 1 owns TMEM.
+//   warps 3-6   softmax group 0 (even tiles), warps 7-10 softmax group 1 (odd
 //               tiles). Each thread owns one query row (= one TMEM lane): it
 //               reads its S row from TMEM, applies the view's mask, keeps a
 //               running max/sum, writes P (bf16 pairs) back into TMEM over
@@ -46,15 +48,14 @@ namespace orthrus {
 
 constexpr int kTileN = 64;          // keys per tile
 constexpr int kTileM = 128;         // query rows per MMA tile
-constexpr int kAttnThreads = 320;   // 10 warps
+constexpr int kAttnThreads = 352;   // 11 warps
 constexpr int kProducerWarp = 0;
-constexpr int kMmaWarp = 1;
-constexpr int kSoftmaxWarp0 = 2;
+constexpr int kMmaWarp0 = 1;        // warps 1 and 2 issue the MMAs of softmax groups 0 and 1
+constexpr int kSoftmaxWarp0 = 3;    // warps 3-6: softmax group 0, warps 7-10: group 1
 constexpr uint32_t kTmemCols = 512;
-constexpr int kSBufs = 3;           // S buffers in TMEM (QK runs this far ahead of PV)
-constexpr uint32_t kTmemS = 0;      // S buffer k at column 64*k
-constexpr uint32_t kTmemO = 192;    // O of group w at column 192 + D*w
-constexpr uint32_t kTmemX = 448;    // (max, sum) exchange between groups, 2 columns a slot
+constexpr int kSPerGroup = 2;       // S buffers per group: QK runs one own tile ahead
+constexpr uint32_t kTmemS = 0;      // S buffer k of group w at column 64*(2w + k)
+constexpr uint32_t kTmemO = 256;    // O of group w at column 256 + D*w
 constexpr float kRescaleLog2 = 8.0f;  // rescale O only when the max grows by > 2^8
 
 struct AttnArgs {
@@ -207,7 +208,7 @@ template <int D>
 struct AttnLayout {
   static constexpr int DH = D / 64;                 // 64-column panels per row
   static constexpr int kNK = (D == 128) ? 5 : 10;   // K ring depth
-  static constexpr int kNV = (D == 128) ? 7 : 14;   // V ring depth
+  static constexpr int kNV = (D == 128) ? 6 : 12;   // V ring depth
   static constexpr int kQPanel = kTileM * 128;      // bytes of one Q panel
   static constexpr int kQBytes = DH * kQPanel;
   static constexpr int kKVPanel = kTileN * 128;        // bytes of one K (or V) panel
@@ -215,7 +216,8 @@ struct AttnLayout {
   static constexpr int kQOff = 0;
   static constexpr int kKOff = kQOff + kQBytes;
   static constexpr int kVOff = kKOff + kNK * kKVBytes;
-  static constexpr int kBarOff = kVOff + kNV * kKVBytes;
+  static constexpr int kXOff = kVOff + kNV * kKVBytes;  // (max, sum) exchange [2][2][128]
+  static constexpr int kBarOff = kXOff + 2 * 2 * kTileM * 8;
   // barrier indices
   static constexpr int kBarKFull = 0;
   static constexpr int kBarKEmpty = kBarKFull + kNK;
@@ -223,19 +225,19 @@ struct AttnLayout {
   static constexpr int kBarVEmpty = kBarVFull + kNV;
   static constexpr int kBarQFull = kBarVEmpty + kNV;
   static constexpr int kBarQEmpty = kBarQFull + 1;
-  static constexpr int kBarSFull = kBarQEmpty + 1;      // [kSBufs]
-  static constexpr int kBarPReady = kBarSFull + kSBufs;  // [2]
+  static constexpr int kBarSFull = kBarQEmpty + 1;             // [2 groups][kSPerGroup]
+  static constexpr int kBarPReady = kBarSFull + 2 * kSPerGroup;  // [2]
   static constexpr int kBarOReady = kBarPReady + 2;      // [2]
   static constexpr int kBarOFree = kBarOReady + 2;
   static constexpr int kBarXchg = kBarOFree + 1;
-  static constexpr int kBarDrain = kBarXchg + 1;
-  static constexpr int kNumBars = kBarDrain + 1;
+  static constexpr int kBarDrain = kBarXchg + 1;  // [2]
+  static constexpr int kNumBars = kBarDrain + 2;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;  // abort flag, TMEM base
   static constexpr int kBytes = kMiscOff + 16;
   static constexpr int kAlloc = kBytes + 1024;  // slack to align the base
   static_assert(kAlloc <= 232448, "shared memory budget exceeded");
-  // QK runs kSBufs tiles ahead of PV: the K ring must hold that many tiles.
-  static_assert(kNK >= kSBufs, "K ring shallower than the QK lead");
+  // Each MMA warp runs QK up to two own tiles (four tiles) ahead of PV.
+  static_assert(kNK >= 4, "K ring shallower than the QK lead");
 };
 
 // Descriptors of the four MMA operands (all SWIZZLE_128B).
@@ -400,14 +402,21 @@ __device__ __forceinline__ bool step_next(const AttnArgs& a, TileStep& s) {
   return true;
 }
 
-// The issuing thread's scalar work sits between consecutive MMAs, so every
-// operand descriptor is a precomputed base plus a compile-time step: the
-// 14-bit start-address field holds (smem address >> 4) and never carries.
+// One MMA warp per softmax group w: it issues QK and PV for the group's tiles
+// (global tile index parity w). The issuing thread's scalar work sits between
+// consecutive MMAs, so every operand descriptor is a precomputed base plus a
+// compile-time step: the 14-bit start-address field holds (smem address >> 4)
+// and never carries.
+//
+// Q bookkeeping covers every segment, own tiles or not: at a segment start the
+// warp waits for that unit's Q tile, and after its last QK of the segment it
+// commits one arrival on q_empty (two arrivals, one per warp, release Q).
+// Waiting for the next Q before committing for it keeps one warp from
+// completing a q_empty phase on its own.
 template <int D>
 __device__ __forceinline__ void mma_role(const AttnArgs& a, uint8_t* smem, uint32_t tmem,
-                                         volatile int* abort_flag) {
+                                         volatile int* abort_flag, int w) {
   using Lay = AttnLayout<D>;
-  const int lane = threadIdx.x & 31;
   const uint32_t base = smem_u32(smem);
   const uint32_t bars = base + Lay::kBarOff;
   constexpr uint32_t kIdescQK = idesc_bf16_f32(kTileM, kTileN, 0);
@@ -415,6 +424,8 @@ __device__ __forceinline__ void mma_role(const AttnArgs& a, uint8_t* smem, uint3
   const uint64_t dq = smem_desc_sw128(base + Lay::kQOff, 16, 1024);
   const uint64_t dk = smem_desc_sw128(base + Lay::kKOff, 16, 1024);
   const uint64_t dv = smem_desc_sw128(base + Lay::kVOff, Lay::kKVPanel, 1024);
+  const uint32_t s_base = tmem + kTmemS + 64u * kSPerGroup * w;
+  const uint32_t o_acc = tmem + kTmemO + (uint32_t)(D * w);
 
   // Every lane polls the barrier (no divergence around the wait); a vote makes
   // the verdict warp-uniform.
@@ -423,15 +434,15 @@ __device__ __forceinline__ void mma_role(const AttnArgs& a, uint8_t* smem, uint3
     return __all_sync(0xffffffffu, ok);
   };
 
-  // S buffer it % 3 is free again once the softmax group has published P for
-  // tile it - 3, which issue_pv of that tile waited for.
-  auto issue_qk = [&](const TileStep& j) -> bool {
+  // QK of own tile m (global tile j) into S buffer m % 2; that buffer last held
+  // P of own tile m - 2, whose PV this warp issued before: the tensor pipe runs
+  // one thread's MMAs in order, so P is read before it is overwritten.
+  auto issue_qk = [&](const TileStep& j, int m) -> bool {
     const int slot = j.it % Lay::kNK;
     if (!wait(bars + 8u * (Lay::kBarKFull + slot), (j.it / Lay::kNK) & 1)) return false;
-    if (j.t == j.sg.t0 && !wait(bars + 8u * Lay::kBarQFull, j.si & 1)) return false;
     tc_fence_after();
-    const int sb = j.it % kSBufs;
-    const uint32_t d = tmem + kTmemS + 64u * sb;
+    const int sb = m & (kSPerGroup - 1);
+    const uint32_t d = s_base + 64u * sb;
     const uint64_t kd = dk + (uint64_t)((slot * Lay::kKVBytes) >> 4);
 #pragma unroll
     for (int kk = 0; kk < D / 16; ++kk) {
@@ -440,25 +451,23 @@ __device__ __forceinline__ void mma_role(const AttnArgs& a, uint8_t* smem, uint3
       if (elect_one()) mma_bf16_ss(d, aq, bk, kIdescQK, kk > 0 ? 1u : 0u);
     }
     if (elect_one()) {
-      mma_commit(bars + 8u * (Lay::kBarSFull + sb));
+      mma_commit(bars + 8u * (Lay::kBarSFull + kSPerGroup * w + sb));
       mma_commit(bars + 8u * (Lay::kBarKEmpty + slot));
-      if (j.t == j.sg.t1 - 1) mma_commit(bars + 8u * Lay::kBarQEmpty);
     }
     __syncwarp();
     return true;
   };
 
-  auto issue_pv = [&](const TileStep& j) -> bool {
-    const int w = j.it & 1;
+  auto issue_pv = [&](const TileStep& j, int m) -> bool {
     const int slot = j.it % Lay::kNV;
     // p_ready also means the tile's V copy has landed: the softmax group waits
     // for it before publishing P, which keeps that wait off this warp's path.
-    if (!wait(bars + 8u * (Lay::kBarPReady + w), (j.it >> 1) & 1)) return false;
-    if (j.t == j.sg.t0 && j.si > 0 && !wait(bars + 8u * Lay::kBarOFree, (j.si - 1) & 1)) return false;
+    if (!wait(bars + 8u * (Lay::kBarPReady + w), m & 1)) return false;
     const int nvalid = tile_valid_keys(j.t, j.L, j.np, j.Kb);
     if (nvalid < kTileN) {
       // Rows past the last valid key may hold stale or non-finite data;
       // P is zero there, but 0 * NaN is NaN, so clear those V rows.
+      const int lane = threadIdx.x & 31;
       const uint32_t v = base + Lay::kVOff + slot * Lay::kKVBytes;
       const int rows = kTileN - nvalid;
       const int chunks = rows * Lay::DH * 8;  // 16-byte chunks
@@ -472,17 +481,13 @@ __device__ __forceinline__ void mma_role(const AttnArgs& a, uint8_t* smem, uint3
       __syncwarp();
     }
     tc_fence_after();
-    // P of this tile sits in the first 32 columns of its S buffer; the next QK
-    // into that buffer is issued after this PV, and the tensor pipe runs one
-    // thread's MMAs in order, so P is read before it is overwritten.
-    const uint32_t pa = tmem + kTmemS + 64u * (j.it % kSBufs);
+    const uint32_t pa = s_base + 64u * (m & (kSPerGroup - 1));
     const uint64_t vd = dv + (uint64_t)((slot * Lay::kKVBytes) >> 4);
-    const uint32_t d = tmem + kTmemO + (uint32_t)(D * w);
     const uint32_t acc0 = (j.t - j.sg.t0 >= 2) ? 1u : 0u;
 #pragma unroll
     for (int kk = 0; kk < kTileN / 16; ++kk) {
       const uint64_t bv = vd + (uint64_t)((kk * 16 * 128) >> 4);
-      if (elect_one()) mma_bf16_ts(d, pa + 8u * kk, bv, kIdescPV, (kk > 0) ? 1u : acc0);
+      if (elect_one()) mma_bf16_ts(o_acc, pa + 8u * kk, bv, kIdescPV, (kk > 0) ? 1u : acc0);
     }
     if (elect_one()) {
       mma_commit(bars + 8u * (Lay::kBarOReady + w));
@@ -492,24 +497,52 @@ __device__ __forceinline__ void mma_role(const AttnArgs& a, uint8_t* smem, uint3
     return true;
   };
 
-  TileStep qs, ps;
+  // QK walk over every tile: Q waits and commits at segment edges, QK for own tiles.
+  TileStep qs;
   cursor_init(a, blockIdx.x, qs.cur);
   qs.si = -1;
   qs.it = -1;
   qs.valid = false;
-  ps = qs;
+  TileStep ps = qs;
+  int mq = 0, mp = 0;  // own tiles issued (QK) / (PV)
   bool ok = true;
-  for (int k = 0; k < kSBufs && ok; ++k)
-    if (step_next(a, qs)) ok = issue_qk(qs);
-  while (ok && step_next(a, ps)) {
-    ok = issue_pv(ps);
-    if (ok && step_next(a, qs)) ok = issue_qk(qs);
-  }
+  auto advance_qk = [&]() -> bool {  // issue the next own QK; false at the end
+    while (ok && step_next(a, qs)) {
+      if (qs.t == qs.sg.t0 && !wait(bars + 8u * Lay::kBarQFull, qs.si & 1)) { ok = false; break; }
+      bool issued = false;
+      if ((qs.it & 1) == w) {
+        if (!issue_qk(qs, mq)) { ok = false; break; }
+        ++mq;
+        issued = true;
+      }
+      if (qs.t == qs.sg.t1 - 1) {
+        if (elect_one()) mma_commit(bars + 8u * Lay::kBarQEmpty);
+        __syncwarp();
+      }
+      if (issued) return true;
+    }
+    return false;
+  };
+  auto advance_pv = [&]() -> bool {
+    while (ok && step_next(a, ps)) {
+      if ((ps.it & 1) != w) continue;
+      if (ps.t <= ps.sg.t0 + 1 && ps.si > 0 &&
+          !wait(bars + 8u * Lay::kBarOFree, (ps.si - 1) & 1)) { ok = false; break; }
+      if (!issue_pv(ps, mp)) { ok = false; break; }
+      ++mp;
+      return true;
+    }
+    return false;
+  };
+  advance_qk();
+  advance_qk();
+  while (ok && advance_pv()) advance_qk();
+  while (ok && advance_qk()) {}  // finish the Q bookkeeping walk
   // Drain: every MMA issued above completes before TMEM is released.
-  if (lane == 0) {
-    mma_commit(bars + 8u * Lay::kBarDrain);
+  if (elect_one()) {
+    mma_commit(bars + 8u * (Lay::kBarDrain + w));
     volatile int no_abort = 0;
-    mbar_wait(bars + 8u * Lay::kBarDrain, 0, &no_abort, 20000000ull);
+    mbar_wait(bars + 8u * (Lay::kBarDrain + w), 0, &no_abort, 20000000ull);
   }
   __syncwarp();
 }
@@ -561,11 +594,11 @@ __device__ __forceinline__ void softmax_role(const AttnArgs& a, uint8_t* smem, u
 
     for (int t = sg.t0; t < sg.t1; ++t, ++it) {
       if ((it & 1) != w) continue;
-      const int sb = it % kSBufs;
-      if (!wait(bar(Lay::kBarSFull + sb), (it / kSBufs) & 1)) { ok = false; break; }
+      const int sb = cnt & (kSPerGroup - 1);  // this group's own tile cnt -> S buffer
+      if (!wait(bar(Lay::kBarSFull + kSPerGroup * w + sb), (cnt / kSPerGroup) & 1)) { ok = false; break; }
       tc_fence_after();
       float s[64];
-      const uint32_t t_s = tmem + lane_off + kTmemS + 64u * sb;
+      const uint32_t t_s = tmem + lane_off + kTmemS + 64u * (kSPerGroup * w + sb);
       tmem_ld32(t_s, *reinterpret_cast<float(*)[32]>(&s[0]));
       tmem_ld32(t_s + 32, *reinterpret_cast<float(*)[32]>(&s[32]));
       tmem_wait_ld();
@@ -645,15 +678,13 @@ __device__ __forceinline__ void softmax_role(const AttnArgs& a, uint8_t* smem, u
       if (!wait(bar(Lay::kBarOReady + w), pv_waited & 1)) { ok = false; break; }
       ++pv_waited;
     }
-    tmem_st2(tmem + lane_off + kTmemX + 2u * ((si & 1) * 2 + w), m_ref, l_sum);
-    tmem_wait_st();
-    tc_fence_before();
+    float2* xch = reinterpret_cast<float2*>(smem + Lay::kXOff);  // [si & 1][group][row]
+    xch[((si & 1) * 2 + w) * kTileM + row] = make_float2(m_ref, l_sum);
     mbar_arrive(bar(Lay::kBarXchg));
     if (!wait(bar(Lay::kBarXchg), si & 1)) { ok = false; break; }
     tc_fence_after();
-    float m_o, l_o;
-    tmem_ld2(tmem + lane_off + kTmemX + 2u * ((si & 1) * 2 + (1 - w)), m_o, l_o);
-    tmem_wait_ld();
+    const float2 other = xch[((si & 1) * 2 + (1 - w)) * kTileM + row];
+    const float m_o = other.x, l_o = other.y;
     const float m0 = w == 0 ? m_ref : m_o, l0 = w == 0 ? l_sum : l_o;
     const float m1 = w == 0 ? m_o : m_ref, l1 = w == 0 ? l_o : l_sum;
     float M = NEG_INF;
@@ -748,8 +779,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(bars + 8u * (Lay::kBarVEmpty + s), 1);
     }
     mbar_init(bars + 8u * Lay::kBarQFull, 1);
-    mbar_init(bars + 8u * Lay::kBarQEmpty, 1);
-    for (int k = 0; k < kSBufs; ++k) mbar_init(bars + 8u * (Lay::kBarSFull + k), 1);
+    mbar_init(bars + 8u * Lay::kBarQEmpty, 2);  // one arrival per MMA warp
+    for (int k = 0; k < 2 * kSPerGroup; ++k) mbar_init(bars + 8u * (Lay::kBarSFull + k), 1);
     for (int w = 0; w < 2; ++w) {
       mbar_init(bars + 8u * (Lay::kBarPReady + w), 128);
       mbar_init(bars + 8u * (Lay::kBarOReady + w), 1);
@@ -757,6 +788,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     mbar_init(bars + 8u * Lay::kBarOFree, 256);
     mbar_init(bars + 8u * Lay::kBarXchg, 256);
     mbar_init(bars + 8u * Lay::kBarDrain, 1);
+    mbar_init(bars + 8u * (Lay::kBarDrain + 1), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -767,7 +799,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     prefetch_tmap(&tm_kb);
     prefetch_tmap(&tm_vb);
   }
-  if (warp == kMmaWarp) {
+  if (warp == kMmaWarp0) {
     tmem_alloc(smem_u32(tmem_slot), kTmemCols);
     tmem_relinquish();
   }
@@ -779,8 +811,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   if (warp == kProducerWarp) {
     if ((threadIdx.x & 31) == 0)
       producer_role<D>(a, smem, &tm_q, &tm_kc, &tm_vc, &tm_kb, &tm_vb, abort_flag);
-  } else if (warp == kMmaWarp) {
-    mma_role<D>(a, smem, tmem, abort_flag);
+  } else if (warp < kSoftmaxWarp0) {
+    mma_role<D>(a, smem, tmem, abort_flag, warp - kMmaWarp0);
   } else {
     softmax_role<D>(a, smem, tmem, abort_flag);
   }
@@ -788,7 +820,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
+  if (warp == kMmaWarp0) tmem_dealloc(tmem, kTmemCols);
   if (threadIdx.x == 0 && *abort_flag) raise_flag(a, ORTHRUS_FLAG_TIMEOUT);
 }
 

@@ -157,7 +157,14 @@ orthrus_status_t plan_attn(const orthrus_attn_params* p, int sms, AttnPlan* pl) 
     pl->chunked = 0;
     pl->chunk_tiles = 0;
     pl->max_chunks = 0;
-    int c = p->max_ctas > 0 ? p->max_ctas : sms;
+    // Balanced ranges over one CTA per SM. When the (sequence, KV head) units
+    // number between 3/4 of the SMs and the SM count, one CTA per unit leaves
+    // a few SMs idle but cuts no unit, which saves the partial/merge work and
+    // the in-CTA unit switches that a near-one-unit range split would add.
+    const long long units = static_cast<long long>(p->B) * p->Hkv;
+    int auto_ctas = sms;
+    if (units >= (3LL * sms) / 4 && units <= sms) auto_ctas = static_cast<int>(units);
+    int c = p->max_ctas > 0 ? p->max_ctas : auto_ctas;
     if (c < 1) c = 1;
     if (c > 65535) c = 65535;
     pl->grid = c;
