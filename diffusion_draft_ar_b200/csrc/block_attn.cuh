@@ -75,6 +75,7 @@ struct AttnArgs {
   int max_chunks;    // chunked: chunks per unit (grid = B * Hkv * max_chunks)
   int num_ctas;      // grid size
   unsigned long long timeout_ns;
+  int fault_inject;  // test hook: 1 drops each CTA's first V copy (a wait must time out)
 };
 
 // ---------------------------------------------------------------------------
@@ -344,6 +345,12 @@ __device__ __forceinline__ void producer_role(const AttnArgs& a, uint8_t* smem,
       ++kt;
       if (vr > 0 && !mbar_wait(bars + 8u * (Lay::kBarVEmpty + vs), (vr - 1) & 1, abort_flag,
                                a.timeout_ns)) { ok = false; break; }
+      if (a.fault_inject == 1 && vt == 0) {
+        // injected fault: this copy is never issued, so its full barrier never
+        // completes and the consumers' bounded waits must give up
+        ++vt;
+        continue;
+      }
       const uint32_t vfb = bars + 8u * (Lay::kBarVFull + vs);
       const uint32_t vdst = base + Lay::kVOff + vs * Lay::kKVBytes;
       mbar_arrive_expect_tx(vfb, bytes);

@@ -243,6 +243,12 @@ orthrus_status_t launch_attn(const orthrus_attn_params* p, const AttnPlan& pl, i
   a.max_chunks = pl.max_chunks;
   a.num_ctas = pl.grid;
   a.timeout_ns = wait_timeout_ns();
+  {
+    // Test hook for failure detection, read on every call: ORTHRUS_FAULT_INJECT=1
+    // withholds one copy per CTA so that a pipeline wait runs out.
+    const char* fi = std::getenv("ORTHRUS_FAULT_INJECT");
+    a.fault_inject = fi ? std::atoi(fi) : 0;
+  }
 
   block_attn_kernel<D><<<pl.grid, kAttnThreads, Lay::kAlloc, stream>>>(tq, tkc, tvc, tkb, tvb, a);
   cudaError_t e = cudaGetLastError();

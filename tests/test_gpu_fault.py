@@ -1,0 +1,57 @@
+"""Failure detection without a GPU fault: a copy the pipeline needs is withheld
+(ORTHRUS_FAULT_INJECT=1), so a bounded wait runs out; the kernel must report
+ORTHRUS_FLAG_TIMEOUT through the error word, return, and leave the CUDA context
+usable for the next, correct call. Runs in a child process so the short wait
+limit (ORTHRUS_WAIT_TIMEOUT_MS, read once per process) stays local to it."""
+import os
+import subprocess
+import sys
+
+import pytest
+
+from tests._gpu import gpu, needs_cuda
+
+pytestmark = [gpu, needs_cuda]
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+CHILD = r'''
+import os, sys, numpy as np, torch
+sys.path.insert(0, ROOT)
+import oracle
+from diffusion_draft_ar_b200 import workloads as W
+from diffusion_draft_ar_b200 import orthrus as O
+from tests._helpers import oracle_attn_args, small_workload
+w = small_workload(name="fault", B=3, Hq=8, Hkv=2, D=128, page_size=64, prefix_len=200, block=8,
+                   paged=True, headroom=64)
+wi = W.WorkloadInputs(w, seed=1)
+m, r = wi.meta, wi.rounds[0]
+d = lambda t: t.cuda()
+args = (d(r.q["verify"]), d(wi.k_cache), d(wi.v_cache), d(r.k_block["verify"]), d(r.v_block["verify"]),
+        d(m.prefix_lens), d(m.cu_block), d(m.page_table))
+out = torch.zeros_like(args[0])
+err = torch.zeros(1, dtype=torch.int32, device="cuda")
+p = O.attn_params("verify", *args, out, w.max_block, max_ctas=4)
+ws = torch.empty(O.block_attn_workspace_size(p), dtype=torch.uint8, device="cuda")
+os.environ["ORTHRUS_FAULT_INJECT"] = "1"
+O.block_attn("verify", *args, out, ws, w.max_block, max_ctas=4, error_flag=err)
+torch.cuda.synchronize()
+flag = int(err.item())
+assert flag & O.FLAG_TIMEOUT, flag
+os.environ["ORTHRUS_FAULT_INJECT"] = "0"
+err.zero_()
+O.block_attn("verify", *args, out, ws, w.max_block, max_ctas=4, error_flag=err)
+torch.cuda.synchronize()
+assert int(err.item()) == 0
+ref = oracle.block_attn(*oracle_attn_args(wi, "verify"))
+e = np.abs(out.double().cpu().numpy() - ref).max()
+assert e <= 2e-2, e
+print("FAULT-OK", flag)
+'''
+
+
+def test_withheld_copy_times_out_and_context_survives():
+    env = dict(os.environ, ORTHRUS_WAIT_TIMEOUT_MS="50", PYTHONPATH=ROOT)
+    r = subprocess.run([sys.executable, "-c", "ROOT = %r\n" % ROOT + CHILD], env=env,
+                       capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stdout + r.stderr
+    assert "FAULT-OK" in r.stdout
