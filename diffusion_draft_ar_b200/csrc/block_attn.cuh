@@ -117,14 +117,41 @@ __device__ __forceinline__ int unit_chunks(const AttnArgs& a, int nt) {
   return c < 1 ? 1 : c;
 }
 
-__device__ __forceinline__ long long total_tiles(const AttnArgs& a) {
-  long long T = 0;
-  for (int b = 0; b < a.B; ++b) T += (long long)a.Hkv * seq_tiles(a, b);
-  return T;
-}
 __device__ __forceinline__ long long range_begin(long long T, int c, int C) {
   return T * c / C;
 }
+
+// What the schedule needs of sequence b: tiles, clamped prefix length, K_b and
+// first block row. The attention kernel computes these once per CTA into a
+// shared-memory table (sequences 0 .. kSeqTableCap-1); later sequences are
+// read from global memory.
+struct SeqInfo {
+  int nt, L, Kb, row0;
+};
+constexpr int kSeqTableCap = 512;
+
+__device__ __forceinline__ SeqInfo seq_info_global(const AttnArgs& a, int b) {
+  SeqInfo s;
+  s.Kb = seq_block_len(a, b);
+  s.L = seq_prefix_len(a, b);
+  s.row0 = seq_row0(a, b);
+  s.nt = s.Kb <= 0 ? 0 : (s.L + kTileN - 1) / kTileN + 1;
+  return s;
+}
+
+struct SeqTable {
+  const int4* rows;  // shared memory, kSeqTableCap entries {nt, L, Kb, row0}
+  __device__ __forceinline__ SeqInfo get(const AttnArgs& a, int b) const {
+    if (b < kSeqTableCap) {
+      const int4 r = rows[b];
+      return SeqInfo{r.x, r.y, r.z, r.w};
+    }
+    return seq_info_global(a, b);
+  }
+  __device__ __forceinline__ int nt(const AttnArgs& a, int b) const {
+    return b < kSeqTableCap ? rows[b].x : seq_info_global(a, b).nt;
+  }
+};
 
 struct Segment {
   int b, h, t0, t1, nt;
@@ -138,49 +165,10 @@ struct SegCursor {
   int cta;
 };
 
-__device__ __forceinline__ void cursor_init(const AttnArgs& a, int cta, SegCursor& c) {
-  c.cta = cta;
-  c.first = 1;
-  c.b = a.B;
-  c.h = 0;
-  c.t = 0;
-  c.remaining = 0;
-  if (a.chunked) {
-    const int chunk = cta % a.max_chunks;
-    const int u = cta / a.max_chunks;
-    const int b = u / a.Hkv;
-    if (b >= a.B) return;
-    const int nt = seq_tiles(a, b);
-    if (nt == 0 || chunk >= unit_chunks(a, nt)) return;
-    c.b = b;
-    c.h = u % a.Hkv;
-    c.t = chunk * a.chunk_tiles;
-    c.remaining = (chunk == unit_chunks(a, nt) - 1) ? (nt - c.t) : a.chunk_tiles;
-    return;
-  }
-  const long long T = total_tiles(a);
-  const long long g0 = range_begin(T, cta, a.num_ctas);
-  c.remaining = range_begin(T, cta + 1, a.num_ctas) - g0;
-  if (c.remaining <= 0) return;
-  long long acc = 0;
-  for (int b = 0; b < a.B; ++b) {
-    const int nt = seq_tiles(a, b);
-    const long long U = (long long)a.Hkv * nt;
-    if (g0 < acc + U) {
-      const long long off = g0 - acc;
-      c.b = b;
-      c.h = (int)(off / nt);
-      c.t = (int)(off % nt);
-      return;
-    }
-    acc += U;
-  }
-  c.remaining = 0;
-}
-
-__device__ __forceinline__ bool cursor_next(const AttnArgs& a, SegCursor& c, Segment& s) {
+__device__ __forceinline__ bool cursor_next(const AttnArgs& a, const SeqTable& tab, SegCursor& c,
+                                            Segment& s) {
   if (c.remaining <= 0 || c.b >= a.B) return false;
-  const int nt = seq_tiles(a, c.b);
+  const int nt = tab.nt(a, c.b);
   long long end = c.t + c.remaining;
   const int t1 = end < nt ? (int)end : nt;
   s.b = c.b;
@@ -197,7 +185,7 @@ __device__ __forceinline__ bool cursor_next(const AttnArgs& a, SegCursor& c, Seg
     c.h = 0;
     do {
       ++c.b;
-    } while (c.b < a.B && seq_tiles(a, c.b) == 0);
+    } while (c.b < a.B && tab.nt(a, c.b) == 0);
   }
   return true;
 }
@@ -221,8 +209,8 @@ struct AttnLayout {
   static constexpr int kBarOff = kXOff + 2 * 2 * kTileM * 8;
   // barrier indices
   static constexpr int kBarKFull = 0;
-  static constexpr int kBarKEmpty = kBarKFull + kNK;
-  static constexpr int kBarVFull = kBarKEmpty + kNK;
+  static constexpr int kBarKEmpty = kBarKFull + kNK;  // [slot][consuming MMA warp]
+  static constexpr int kBarVFull = kBarKEmpty + 2 * kNK;
   static constexpr int kBarVEmpty = kBarVFull + kNV;
   static constexpr int kBarQFull = kBarVEmpty + kNV;
   static constexpr int kBarQEmpty = kBarQFull + 1;
@@ -234,12 +222,37 @@ struct AttnLayout {
   static constexpr int kBarDrain = kBarXchg + 1;  // [2]
   static constexpr int kNumBars = kBarDrain + 2;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;  // abort flag, TMEM base
-  static constexpr int kBytes = kMiscOff + 16;
+  // schedule: start cursor {b, h, t, -, remaining}, scan scratch, sequence table
+  static constexpr int kSchedOff = (kMiscOff + 16 + 15) / 16 * 16;
+  static constexpr int kScanOff = kSchedOff + 32;
+  static constexpr int kSeqOff = kScanOff + 16 * 8;
+  static constexpr int kBytes = kSeqOff + kSeqTableCap * 16;
   static constexpr int kAlloc = kBytes + 1024;  // slack to align the base
   static_assert(kAlloc <= 232448, "shared memory budget exceeded");
   // Each MMA warp runs QK up to two own tiles (four tiles) ahead of PV.
   static_assert(kNK >= 4, "K ring shallower than the QK lead");
 };
+
+// K slot s releases. Fill k of slot s holds tile s + k*kNK, whose QK is issued
+// by MMA warp (tile & 1), and that warp commits the release on its own
+// barrier K_empty[s][warp]: every commit-fed barrier is fed by one thread.
+// With an odd ring depth the consuming warp alternates from fill to fill.
+template <int D>
+__device__ __forceinline__ int kslot_warp(int s, int k) {
+  return (s + k * AttnLayout<D>::kNK) & 1;
+}
+// Releases of K_empty[s][w] that precede fill k's release (fill k has warp w).
+template <int D>
+__device__ __forceinline__ int kslot_phase(int k) {
+  return (AttnLayout<D>::kNK & 1) ? (k >> 1) : k;
+}
+// Releases that K_empty[s][w] receives from fills 0 .. n-1 of slot s.
+template <int D>
+__device__ __forceinline__ int kslot_releases(int s, int w, int n) {
+  if (!(AttnLayout<D>::kNK & 1)) return (s & 1) == w ? n : 0;
+  const int k0 = (w - s) & 1;  // first fill consumed by warp w
+  return n > k0 ? (n - k0 + 1) >> 1 : 0;
+}
 
 // Descriptors of the four MMA operands (all SWIZZLE_128B).
 // A = Q (K-major): panel p at +p*kQPanel, 8-row groups 1024 B apart.
@@ -272,6 +285,115 @@ __device__ __forceinline__ void raise_flag(const AttnArgs& a, int bits) {
 }
 
 // ---------------------------------------------------------------------------
+// Schedule prologue, run by the whole CTA before the roles split: the
+// per-sequence facts are loaded in parallel into the shared table, a block
+// reduction gives the total tile count T, and a block scan over the sequences'
+// tile counts finds the unit and tile where this CTA's range starts. Returns
+// false (uniformly) when the range is empty.
+__device__ __forceinline__ long long block_sum_ll(long long x, long long* scan) {
+  constexpr int kWarps = kAttnThreads / 32;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  if ((threadIdx.x & 31) == 0) scan[threadIdx.x >> 5] = x;
+  __syncthreads();
+  long long t = 0;
+#pragma unroll
+  for (int k = 0; k < kWarps; ++k) t += scan[k];
+  __syncthreads();
+  return t;
+}
+
+template <int D>
+__device__ __forceinline__ bool schedule_prologue(const AttnArgs& a, uint8_t* smem,
+                                                  SeqTable& tab, SegCursor& start) {
+  using Lay = AttnLayout<D>;
+  constexpr int kWarps = kAttnThreads / 32;
+  int* sc = reinterpret_cast<int*>(smem + Lay::kSchedOff);  // b, h, t
+  long long* srem = reinterpret_cast<long long*>(smem + Lay::kSchedOff + 16);
+  long long* scan = reinterpret_cast<long long*>(smem + Lay::kScanOff);
+  int4* rows = reinterpret_cast<int4*>(smem + Lay::kSeqOff);
+  tab.rows = rows;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+  long long part = 0;
+  for (int b = tid; b < a.B; b += kAttnThreads) {
+    const SeqInfo si = seq_info_global(a, b);
+    if (b < kSeqTableCap) rows[b] = make_int4(si.nt, si.L, si.Kb, si.row0);
+    part += (long long)a.Hkv * si.nt;
+  }
+  const long long T = block_sum_ll(part, scan);  // also publishes the table
+
+  if (a.chunked) {
+    if (tid == 0) {
+      int b = a.B, h = 0, t = 0;
+      long long rem = 0;
+      const int chunk = blockIdx.x % a.max_chunks;
+      const int u = blockIdx.x / a.max_chunks;
+      const int bu = u / a.Hkv;
+      if (bu < a.B) {
+        const int nt = tab.nt(a, bu);
+        if (nt > 0 && chunk < unit_chunks(a, nt)) {
+          b = bu;
+          h = u % a.Hkv;
+          t = chunk * a.chunk_tiles;
+          rem = (chunk == unit_chunks(a, nt) - 1) ? (nt - t) : a.chunk_tiles;
+        }
+      }
+      sc[0] = b, sc[1] = h, sc[2] = t;
+      *srem = rem;
+    }
+  } else {
+    const long long g0 = range_begin(T, blockIdx.x, a.num_ctas);
+    const long long rem = range_begin(T, blockIdx.x + 1, a.num_ctas) - g0;
+    if (tid == 0) {
+      sc[0] = a.B, sc[1] = 0, sc[2] = 0;
+      *srem = rem;
+    }
+    if (rem > 0) {
+      long long off = 0;  // tiles of the sequences before this chunk of them
+      for (int base = 0; base < a.B; base += kAttnThreads) {
+        const int b = base + tid;
+        const int nt = b < a.B ? tab.nt(a, b) : 0;
+        const long long n = (long long)a.Hkv * nt;
+        long long x = n;  // inclusive scan within the warp
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const long long y = __shfl_up_sync(0xffffffffu, x, o);
+          if (lane >= o) x += y;
+        }
+        if (lane == 31) scan[warp] = x;
+        __syncthreads();
+        long long before = 0, total = 0;
+#pragma unroll
+        for (int k = 0; k < kWarps; ++k) {
+          const long long v = scan[k];
+          before += (k < warp) ? v : 0;
+          total += v;
+        }
+        const long long excl = off + before + x - n;
+        if (n > 0 && excl <= g0 && g0 < excl + n) {
+          sc[0] = b;
+          sc[1] = (int)((g0 - excl) / nt);
+          sc[2] = (int)((g0 - excl) % nt);
+        }
+        off += total;
+        __syncthreads();
+        if (off > g0) break;
+      }
+    }
+  }
+  __syncthreads();
+  start.cta = blockIdx.x;
+  start.first = 1;
+  start.b = sc[0];
+  start.h = sc[1];
+  start.t = sc[2];
+  start.remaining = *srem;
+  if (start.b >= a.B) start.remaining = 0;
+  return start.remaining > 0;
+}
+
+// ---------------------------------------------------------------------------
 // Roles
 
 // One thread issues everything: the Q tile of each unit, then per key tile its
@@ -283,7 +405,8 @@ template <int D>
 __device__ __forceinline__ void producer_role(const AttnArgs& a, uint8_t* smem,
                                               const CUtensorMap* tm_q, const CUtensorMap* tm_kc,
                                               const CUtensorMap* tm_vc, const CUtensorMap* tm_kb,
-                                              const CUtensorMap* tm_vb, volatile int* abort_flag) {
+                                              const CUtensorMap* tm_vb, volatile int* abort_flag,
+                                              const SeqTable& tab, const SegCursor& start) {
   using Lay = AttnLayout<D>;
   const uint32_t base = smem_u32(smem);
   const uint32_t bars = base + Lay::kBarOff;
@@ -292,14 +415,14 @@ __device__ __forceinline__ void producer_role(const AttnArgs& a, uint8_t* smem,
   int kt = 0, vt = 0, q_issued = 0;  // K copies, V copies and Q tiles issued
   bool ok = true;
 
-  SegCursor cur;
-  cursor_init(a, blockIdx.x, cur);
+  SegCursor cur = start;
   Segment sg;
   int si = 0;
-  while (ok && cursor_next(a, cur, sg)) {
+  while (ok && cursor_next(a, tab, cur, sg)) {
     const int b = sg.b, h = sg.h;
-    const int row0 = seq_row0(a, b);
-    const int L = seq_prefix_len(a, b);
+    const SeqInfo sq = tab.get(a, b);
+    const int row0 = sq.row0;
+    const int L = sq.L;
     const int np = (L + kTileN - 1) / kTileN;
     const int* ptab = a.page_table + (long long)b * a.max_pages;
     // Q tile of this unit: rows (i, g) for i < max_block, g < G.
@@ -330,7 +453,8 @@ __device__ __forceinline__ void producer_role(const AttnArgs& a, uint8_t* smem,
       }
       const uint32_t bytes = block ? blk_bytes : (uint32_t)Lay::kKVBytes;
       // K into its ring (freed by the tile's QK), V into the deeper V ring (freed by PV)
-      if (kr > 0 && !mbar_wait(bars + 8u * (Lay::kBarKEmpty + ks), (kr - 1) & 1, abort_flag,
+      if (kr > 0 && !mbar_wait(bars + 8u * (Lay::kBarKEmpty + 2 * ks + kslot_warp<D>(ks, kr - 1)),
+                               kslot_phase<D>(kr - 1) & 1, abort_flag,
                                a.timeout_ns)) { ok = false; break; }
       const uint32_t kfb = bars + 8u * (Lay::kBarKFull + ks);
       const uint32_t kdst = base + Lay::kKOff + ks * Lay::kKVBytes;
@@ -365,6 +489,29 @@ __device__ __forceinline__ void producer_role(const AttnArgs& a, uint8_t* smem,
     }
     ++si;
   }
+  if (ok && !*abort_flag) {
+    // Producer tail. The MMA warps release K, V and Q slots with
+    // tcgen05.commit, whose mbarrier arrivals land asynchronously; the last
+    // release of each slot is never waited for above. Wait for it, so that no
+    // arrival is still in flight when the CTA exits: it would land on the
+    // barriers of the next CTA that this SM runs, in the same shared memory.
+    for (int s = 0; s < Lay::kNK && ok; ++s) {
+      const int n = kt / Lay::kNK + (s < kt % Lay::kNK ? 1 : 0);
+      for (int w = 0; w < 2 && ok; ++w) {
+        const int r = kslot_releases<D>(s, w, n);
+        if (r > 0)
+          ok = mbar_wait(bars + 8u * (Lay::kBarKEmpty + 2 * s + w), (r - 1) & 1, abort_flag,
+                         a.timeout_ns);
+      }
+    }
+    for (int s = 0; s < Lay::kNV && ok; ++s) {
+      const int n = vt / Lay::kNV + (s < vt % Lay::kNV ? 1 : 0);
+      if (n > 0)
+        ok = mbar_wait(bars + 8u * (Lay::kBarVEmpty + s), (n - 1) & 1, abort_flag, a.timeout_ns);
+    }
+    if (ok && q_issued > 0)
+      ok = mbar_wait(bars + 8u * Lay::kBarQEmpty, (q_issued - 1) & 1, abort_flag, a.timeout_ns);
+  }
   if (!ok || *abort_flag) {
     // Wind down: let every copy this thread started land before the CTA exits.
     volatile int no_abort = 0;
@@ -389,22 +536,23 @@ struct TileStep {
   bool valid;
 };
 
-__device__ __forceinline__ bool step_next(const AttnArgs& a, TileStep& s) {
+__device__ __forceinline__ bool step_next(const AttnArgs& a, const SeqTable& tab, TileStep& s) {
   if (s.valid && s.t + 1 < s.sg.t1) {
     ++s.t;
     ++s.it;
     return true;
   }
-  if (!cursor_next(a, s.cur, s.sg)) {
+  if (!cursor_next(a, tab, s.cur, s.sg)) {
     s.valid = false;
     return false;
   }
   ++s.si;
   ++s.it;
   s.t = s.sg.t0;
-  s.L = seq_prefix_len(a, s.sg.b);
+  const SeqInfo sq = tab.get(a, s.sg.b);
+  s.L = sq.L;
   s.np = (s.L + kTileN - 1) / kTileN;
-  s.Kb = seq_block_len(a, s.sg.b);
+  s.Kb = sq.Kb;
   s.valid = true;
   return true;
 }
@@ -422,7 +570,8 @@ __device__ __forceinline__ bool step_next(const AttnArgs& a, TileStep& s) {
 // completing a q_empty phase on its own.
 template <int D>
 __device__ __forceinline__ void mma_role(const AttnArgs& a, uint8_t* smem, uint32_t tmem,
-                                         volatile int* abort_flag, int w) {
+                                         volatile int* abort_flag, int w, const SeqTable& tab,
+                                         const SegCursor& start) {
   using Lay = AttnLayout<D>;
   const uint32_t base = smem_u32(smem);
   const uint32_t bars = base + Lay::kBarOff;
@@ -459,7 +608,7 @@ __device__ __forceinline__ void mma_role(const AttnArgs& a, uint8_t* smem, uint3
     }
     if (elect_one()) {
       mma_commit(bars + 8u * (Lay::kBarSFull + kSPerGroup * w + sb));
-      mma_commit(bars + 8u * (Lay::kBarKEmpty + slot));
+      mma_commit(bars + 8u * (Lay::kBarKEmpty + 2 * slot + w));
     }
     __syncwarp();
     return true;
@@ -506,7 +655,7 @@ __device__ __forceinline__ void mma_role(const AttnArgs& a, uint8_t* smem, uint3
 
   // QK walk over every tile: Q waits and commits at segment edges, QK for own tiles.
   TileStep qs;
-  cursor_init(a, blockIdx.x, qs.cur);
+  qs.cur = start;
   qs.si = -1;
   qs.it = -1;
   qs.valid = false;
@@ -514,7 +663,7 @@ __device__ __forceinline__ void mma_role(const AttnArgs& a, uint8_t* smem, uint3
   int mq = 0, mp = 0;  // own tiles issued (QK) / (PV)
   bool ok = true;
   auto advance_qk = [&]() -> bool {  // issue the next own QK; false at the end
-    while (ok && step_next(a, qs)) {
+    while (ok && step_next(a, tab, qs)) {
       if (qs.t == qs.sg.t0 && !wait(bars + 8u * Lay::kBarQFull, qs.si & 1)) { ok = false; break; }
       bool issued = false;
       if ((qs.it & 1) == w) {
@@ -531,7 +680,7 @@ __device__ __forceinline__ void mma_role(const AttnArgs& a, uint8_t* smem, uint3
     return false;
   };
   auto advance_pv = [&]() -> bool {
-    while (ok && step_next(a, ps)) {
+    while (ok && step_next(a, tab, ps)) {
       if ((ps.it & 1) != w) continue;
       if (ps.t <= ps.sg.t0 + 1 && ps.si > 0 &&
           !wait(bars + 8u * Lay::kBarOFree, (ps.si - 1) & 1)) { ok = false; break; }
@@ -556,7 +705,8 @@ __device__ __forceinline__ void mma_role(const AttnArgs& a, uint8_t* smem, uint3
 
 template <int D>
 __device__ __forceinline__ void softmax_role(const AttnArgs& a, uint8_t* smem, uint32_t tmem,
-                                             volatile int* abort_flag) {
+                                             volatile int* abort_flag, const SeqTable& tab,
+                                             const SegCursor& start) {
   using Lay = AttnLayout<D>;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -580,15 +730,15 @@ __device__ __forceinline__ void softmax_role(const AttnArgs& a, uint8_t* smem, u
   int cnt = 0;        // tiles this group processed (CTA-wide)
   int pv_waited = 0;  // PV completions of this group already observed
 
-  SegCursor cur;
-  cursor_init(a, blockIdx.x, cur);
+  SegCursor cur = start;
   Segment sg;
   int it = 0, si = 0;
   bool ok = true;
-  while (ok && cursor_next(a, cur, sg)) {
+  while (ok && cursor_next(a, tab, cur, sg)) {
     const int b = sg.b, h = sg.h;
-    const int Kb = seq_block_len(a, b), row0 = seq_row0(a, b);
-    const int L = seq_prefix_len(a, b);
+    const SeqInfo sq = tab.get(a, b);
+    const int Kb = sq.Kb, row0 = sq.row0;
+    const int L = sq.L;
     const int np = (L + kTileN - 1) / kTileN;
     const int rows_valid = a.G * Kb;
     const bool my_valid = row < rows_valid;
@@ -769,17 +919,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   pdl_launch_dependents();
 
   // A CTA whose range is empty has nothing to set up.
-  {
-    SegCursor cur;
-    cursor_init(a, blockIdx.x, cur);
-    if (cur.remaining <= 0 || cur.b >= a.B) return;
-  }
+  SeqTable tab;
+  SegCursor start;
+  if (!schedule_prologue<D>(a, smem, tab, start)) return;
 
   if (threadIdx.x == 0) {
     const uint32_t bars = smem_u32(smem) + Lay::kBarOff;
     for (int s = 0; s < Lay::kNK; ++s) {
       mbar_init(bars + 8u * (Lay::kBarKFull + s), 1);
-      mbar_init(bars + 8u * (Lay::kBarKEmpty + s), 1);
+      mbar_init(bars + 8u * (Lay::kBarKEmpty + 2 * s), 1);
+      mbar_init(bars + 8u * (Lay::kBarKEmpty + 2 * s + 1), 1);
     }
     for (int s = 0; s < Lay::kNV; ++s) {
       mbar_init(bars + 8u * (Lay::kBarVFull + s), 1);
@@ -817,11 +966,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   if (warp == kProducerWarp) {
     if ((threadIdx.x & 31) == 0)
-      producer_role<D>(a, smem, &tm_q, &tm_kc, &tm_vc, &tm_kb, &tm_vb, abort_flag);
+      producer_role<D>(a, smem, &tm_q, &tm_kc, &tm_vc, &tm_kb, &tm_vb, abort_flag, tab, start);
   } else if (warp < kSoftmaxWarp0) {
-    mma_role<D>(a, smem, tmem, abort_flag, warp - kMmaWarp0);
+    mma_role<D>(a, smem, tmem, abort_flag, warp - kMmaWarp0, tab, start);
   } else {
-    softmax_role<D>(a, smem, tmem, abort_flag);
+    softmax_role<D>(a, smem, tmem, abort_flag, tab, start);
   }
 
   tc_fence_before();
