@@ -17,10 +17,10 @@
 // kernel from per-CTA partials (max, sum, normalised accumulator).
 //
 // Roles (352 threads):
-//   warp 0      TMA producer: Q tile per unit; K tiles into a K ring and V
-//               tiles into a separate, deeper V ring (K is released by its
-//               QK three tiles before V is released by its PV); the next
-//               page id is fetched while the current tile's copies are issued.
+//   warp 0      TMA producer, two lanes: lane 0 issues the Q tile per unit
+//               and the K tiles into a K ring, lane 1 the V tiles into a
+//               separate, deeper V ring (K is released by its QK three tiles
+//               before V is released by its PV); both step one tile at a time.
 //   warps 1-2   MMA issuers, one per softmax group: S = Q K^T for the group's
 //               tiles into its two TMEM S buffers (one own tile ahead), and
 //               O += P V into its TMEM accumulator. Two issuing warps overlap
@@ -196,7 +196,7 @@ __device__ __forceinline__ bool cursor_next(const AttnArgs& a, const SeqTable& t
 template <int D>
 struct AttnLayout {
   static constexpr int DH = D / 64;                 // 64-column panels per row
-  static constexpr int kNK = (D == 128) ? 5 : 10;   // K ring depth
+  static constexpr int kNK = (D == 128) ? 4 : 10;   // K ring depth
   static constexpr int kNV = (D == 128) ? 6 : 12;   // V ring depth
   static constexpr int kQPanel = kTileM * 128;      // bytes of one Q panel
   static constexpr int kQBytes = DH * kQPanel;
@@ -209,8 +209,8 @@ struct AttnLayout {
   static constexpr int kBarOff = kXOff + 2 * 2 * kTileM * 8;
   // barrier indices
   static constexpr int kBarKFull = 0;
-  static constexpr int kBarKEmpty = kBarKFull + kNK;  // [slot][consuming MMA warp]
-  static constexpr int kBarVFull = kBarKEmpty + 2 * kNK;
+  static constexpr int kBarKEmpty = kBarKFull + kNK;
+  static constexpr int kBarVFull = kBarKEmpty + kNK;
   static constexpr int kBarVEmpty = kBarVFull + kNV;
   static constexpr int kBarQFull = kBarVEmpty + kNV;
   static constexpr int kBarQEmpty = kBarQFull + 1;
@@ -231,28 +231,15 @@ struct AttnLayout {
   static_assert(kAlloc <= 232448, "shared memory budget exceeded");
   // Each MMA warp runs QK up to two own tiles (four tiles) ahead of PV.
   static_assert(kNK >= 4, "K ring shallower than the QK lead");
+  // Tile it goes to ring slot it % depth and belongs to MMA warp / softmax
+  // group it & 1. With even depths every fill of a slot belongs to the same
+  // consumer, which therefore waits on each phase of that slot's barriers in
+  // turn. With an odd depth a consumer would skip the other consumer's fill
+  // and wait two phases ahead; copies complete out of order, so that fill
+  // could still be in flight and the parity wait would pass early (stale K,
+  // and a release committed before the copy landed).
+  static_assert(kNK % 2 == 0 && kNV % 2 == 0, "ring depths must be even");
 };
-
-// K slot s releases. Fill k of slot s holds tile s + k*kNK, whose QK is issued
-// by MMA warp (tile & 1), and that warp commits the release on its own
-// barrier K_empty[s][warp]: every commit-fed barrier is fed by one thread.
-// With an odd ring depth the consuming warp alternates from fill to fill.
-template <int D>
-__device__ __forceinline__ int kslot_warp(int s, int k) {
-  return (s + k * AttnLayout<D>::kNK) & 1;
-}
-// Releases of K_empty[s][w] that precede fill k's release (fill k has warp w).
-template <int D>
-__device__ __forceinline__ int kslot_phase(int k) {
-  return (AttnLayout<D>::kNK & 1) ? (k >> 1) : k;
-}
-// Releases that K_empty[s][w] receives from fills 0 .. n-1 of slot s.
-template <int D>
-__device__ __forceinline__ int kslot_releases(int s, int w, int n) {
-  if (!(AttnLayout<D>::kNK & 1)) return (s & 1) == w ? n : 0;
-  const int k0 = (w - s) & 1;  // first fill consumed by warp w
-  return n > k0 ? (n - k0 + 1) >> 1 : 0;
-}
 
 // Descriptors of the four MMA operands (all SWIZZLE_128B).
 // A = Q (K-major): panel p at +p*kQPanel, 8-row groups 1024 B apart.
@@ -396,11 +383,15 @@ __device__ __forceinline__ bool schedule_prologue(const AttnArgs& a, uint8_t* sm
 // ---------------------------------------------------------------------------
 // Roles
 
-// One thread issues everything: the Q tile of each unit, then per key tile its
-// K copy into the K ring and its V copy into the V ring (one 3-D box each: 64
-// tokens x both 64-column halves of D, landing as the two swizzled panels the
-// MMA descriptors expect). The next page id is read while the current tile's
-// copies are issued.
+// Two lanes of the producer warp issue every copy: lane 0 the Q tile of each
+// unit and the K tiles into the K ring, lane 1 the V tiles into the V ring.
+// Each key tile is one 3-D box per tensor (64 tokens x both 64-column halves
+// of D, landing as the two swizzled panels the MMA descriptors expect). A box
+// issue holds its thread for a few hundred cycles, so one thread issuing both
+// copies plus the page lookup paced the whole pipeline; the two lanes wait
+// for their ring slots and issue their boxes side by side, one tile per step.
+// Page ids are read four tiles ahead into registers, and the slot and the row
+// inside the page are tracked incrementally (no division per tile).
 template <int D>
 __device__ __forceinline__ void producer_role(const AttnArgs& a, uint8_t* smem,
                                               const CUtensorMap* tm_q, const CUtensorMap* tm_kc,
@@ -408,11 +399,21 @@ __device__ __forceinline__ void producer_role(const AttnArgs& a, uint8_t* smem,
                                               const CUtensorMap* tm_vb, volatile int* abort_flag,
                                               const SeqTable& tab, const SegCursor& start) {
   using Lay = AttnLayout<D>;
+  constexpr unsigned kPair = 0x3u;  // lanes 0 (K) and 1 (V)
+  const bool is_v = (threadIdx.x & 31) == 1;
+  const int depth = is_v ? Lay::kNV : Lay::kNK;
   const uint32_t base = smem_u32(smem);
   const uint32_t bars = base + Lay::kBarOff;
+  const uint32_t ring = base + (is_v ? Lay::kVOff : Lay::kKOff);
+  const uint32_t full0 = bars + 8u * (is_v ? Lay::kBarVFull : Lay::kBarKFull);
+  const uint32_t empty0 = bars + 8u * (is_v ? Lay::kBarVEmpty : Lay::kBarKEmpty);
+  const CUtensorMap* tm_cache = is_v ? tm_vc : tm_kc;
+  const CUtensorMap* tm_blk = is_v ? tm_vb : tm_kb;
   const uint32_t blk_bytes = Lay::DH * a.blk_box_rows * 128;
   const int tiles_per_page = a.page_size / kTileN;
-  int kt = 0, vt = 0, q_issued = 0;  // K copies, V copies and Q tiles issued
+  const int slab_rows = a.Hkv * a.page_size;  // cache rows per page
+  int n = 0, q_issued = 0;  // copies issued into this lane's ring; Q tiles issued
+  int s = 0, r = 0;         // ring slot of copy n and how often it was filled before
   bool ok = true;
 
   SegCursor cur = start;
@@ -422,108 +423,101 @@ __device__ __forceinline__ void producer_role(const AttnArgs& a, uint8_t* smem,
     const int b = sg.b, h = sg.h;
     const SeqInfo sq = tab.get(a, b);
     const int row0 = sq.row0;
-    const int L = sq.L;
-    const int np = (L + kTileN - 1) / kTileN;
+    const int np = (sq.L + kTileN - 1) / kTileN;
     const int* ptab = a.page_table + (long long)b * a.max_pages;
-    // Q tile of this unit: rows (i, g) for i < max_block, g < G.
-    if (si > 0 && !mbar_wait(bars + 8u * Lay::kBarQEmpty, (si - 1) & 1, abort_flag, a.timeout_ns)) {
+    // Q tile of this unit (rows (i, g) for i < max_block, g < G), by lane 0.
+    bool qok = true;
+    if (!is_v && si > 0)
+      qok = mbar_wait(bars + 8u * Lay::kBarQEmpty, (si - 1) & 1, abort_flag, a.timeout_ns);
+    if (!__all_sync(kPair, qok)) {
       ok = false;
       break;
     }
-    mbar_arrive_expect_tx(bars + 8u * Lay::kBarQFull, Lay::DH * a.G * a.q_box_rows * 128);
+    if (!is_v) {
+      mbar_arrive_expect_tx(bars + 8u * Lay::kBarQFull, Lay::DH * a.G * a.q_box_rows * 128);
 #pragma unroll
-    for (int p = 0; p < Lay::DH; ++p)
-      tma_load_3d(base + Lay::kQOff + p * Lay::kQPanel, tm_q, bars + 8u * Lay::kBarQFull, p * 64,
-                  h * a.G, row0);
+      for (int p = 0; p < Lay::DH; ++p)
+        tma_load_3d(base + Lay::kQOff + p * Lay::kQPanel, tm_q, bars + 8u * Lay::kBarQFull,
+                    p * 64, h * a.G, row0);
+    }
     ++q_issued;
-    int page_next = (sg.t0 < np) ? ptab[sg.t0 / tiles_per_page] : 0;
+    // Page ids of the next four prefix tiles and the position of tile t0 in
+    // its page; ahead_* is the page position of tile t + 4.
+    const int t1p = sg.t1 < np ? sg.t1 : np;
+    int sub = sg.t0 % tiles_per_page;
+    int ahead_pidx = sg.t0 / tiles_per_page, ahead_sub = sub;
+    int pq[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      pq[k] = (sg.t0 + k < t1p) ? ptab[ahead_pidx] : 0;
+      if (++ahead_sub == tiles_per_page) ahead_sub = 0, ++ahead_pidx;
+    }
     for (int t = sg.t0; t < sg.t1; ++t) {
-      const int ks = kt % Lay::kNK, kr = kt / Lay::kNK;
-      const int vs = vt % Lay::kNV, vr = vt / Lay::kNV;
       const bool block = t >= np;
       int row = row0;
       if (!block) {
-        int page = page_next;
-        if (t + 1 < np) page_next = ptab[(t + 1) / tiles_per_page];
+        int page = pq[0];
         if (page < 0 || page >= a.num_pages) {
           raise_flag(a, ORTHRUS_FLAG_BAD_PAGE);
           page = 0;  // keep the pipeline flowing on an in-bounds page
         }
-        row = (page * a.Hkv + h) * a.page_size + (t % tiles_per_page) * kTileN;
+        row = page * slab_rows + h * a.page_size + sub * kTileN;
       }
-      const uint32_t bytes = block ? blk_bytes : (uint32_t)Lay::kKVBytes;
-      // K into its ring (freed by the tile's QK), V into the deeper V ring (freed by PV)
-      if (kr > 0 && !mbar_wait(bars + 8u * (Lay::kBarKEmpty + 2 * ks + kslot_warp<D>(ks, kr - 1)),
-                               kslot_phase<D>(kr - 1) & 1, abort_flag,
-                               a.timeout_ns)) { ok = false; break; }
-      const uint32_t kfb = bars + 8u * (Lay::kBarKFull + ks);
-      const uint32_t kdst = base + Lay::kKOff + ks * Lay::kKVBytes;
-      mbar_arrive_expect_tx(kfb, bytes);
-      if (block) {
+      pq[0] = pq[1];
+      pq[1] = pq[2];
+      pq[2] = pq[3];
+      pq[3] = (t + 4 < t1p) ? ptab[ahead_pidx] : 0;
+      if (++ahead_sub == tiles_per_page) ahead_sub = 0, ++ahead_pidx;
+      if (++sub == tiles_per_page) sub = 0;
+      // The slot's previous fill must have been consumed.
+      bool wok = true;
+      if (r > 0) {
+        wok = mbar_wait(empty0 + 8u * s, (r - 1) & 1, abort_flag, a.timeout_ns);
+      }
+      if (!__all_sync(kPair, wok)) {
+        ok = false;
+        break;
+      }
+      // test hook: the first V copy is never issued, so its full barrier never
+      // completes and the consumers' bounded waits must give up
+      if (!(is_v && a.fault_inject == 1 && n == 0)) {
+        const uint32_t fb = full0 + 8u * s;
+        const uint32_t dst = ring + s * Lay::kKVBytes;
+        mbar_arrive_expect_tx(fb, block ? blk_bytes : (uint32_t)Lay::kKVBytes);
+        if (block) {
 #pragma unroll
-        for (int p = 0; p < Lay::DH; ++p)
-          tma_load_3d(kdst + p * Lay::kKVPanel, tm_kb, kfb, p * 64, h, row);
-      } else {
-        tma_load_3d(kdst, tm_kc, kfb, 0, row, 0);
+          for (int p = 0; p < Lay::DH; ++p)
+            tma_load_3d(dst + p * Lay::kKVPanel, tm_blk, fb, p * 64, h, row);
+        } else {
+          tma_load_3d(dst, tm_cache, fb, 0, row, 0);
+        }
       }
-      ++kt;
-      if (vr > 0 && !mbar_wait(bars + 8u * (Lay::kBarVEmpty + vs), (vr - 1) & 1, abort_flag,
-                               a.timeout_ns)) { ok = false; break; }
-      if (a.fault_inject == 1 && vt == 0) {
-        // injected fault: this copy is never issued, so its full barrier never
-        // completes and the consumers' bounded waits must give up
-        ++vt;
-        continue;
-      }
-      const uint32_t vfb = bars + 8u * (Lay::kBarVFull + vs);
-      const uint32_t vdst = base + Lay::kVOff + vs * Lay::kKVBytes;
-      mbar_arrive_expect_tx(vfb, bytes);
-      if (block) {
-#pragma unroll
-        for (int p = 0; p < Lay::DH; ++p)
-          tma_load_3d(vdst + p * Lay::kKVPanel, tm_vb, vfb, p * 64, h, row);
-      } else {
-        tma_load_3d(vdst, tm_vc, vfb, 0, row, 0);
-      }
-      ++vt;
+      ++n;
+      if (++s == depth) s = 0, ++r;
     }
     ++si;
   }
   if (ok && !*abort_flag) {
-    // Producer tail. The MMA warps release K, V and Q slots with
+    // Producer tail. The MMA warps release ring and Q slots with
     // tcgen05.commit, whose mbarrier arrivals land asynchronously; the last
     // release of each slot is never waited for above. Wait for it, so that no
     // arrival is still in flight when the CTA exits: it would land on the
     // barriers of the next CTA that this SM runs, in the same shared memory.
-    for (int s = 0; s < Lay::kNK && ok; ++s) {
-      const int n = kt / Lay::kNK + (s < kt % Lay::kNK ? 1 : 0);
-      for (int w = 0; w < 2 && ok; ++w) {
-        const int r = kslot_releases<D>(s, w, n);
-        if (r > 0)
-          ok = mbar_wait(bars + 8u * (Lay::kBarKEmpty + 2 * s + w), (r - 1) & 1, abort_flag,
-                         a.timeout_ns);
-      }
+    for (int ss = 0; ss < depth && ok; ++ss) {
+      const int nf = n / depth + (ss < n % depth ? 1 : 0);  // fills of slot ss
+      if (nf > 0) ok = mbar_wait(empty0 + 8u * ss, (nf - 1) & 1, abort_flag, a.timeout_ns);
     }
-    for (int s = 0; s < Lay::kNV && ok; ++s) {
-      const int n = vt / Lay::kNV + (s < vt % Lay::kNV ? 1 : 0);
-      if (n > 0)
-        ok = mbar_wait(bars + 8u * (Lay::kBarVEmpty + s), (n - 1) & 1, abort_flag, a.timeout_ns);
-    }
-    if (ok && q_issued > 0)
+    if (!is_v && ok && q_issued > 0)
       ok = mbar_wait(bars + 8u * Lay::kBarQEmpty, (q_issued - 1) & 1, abort_flag, a.timeout_ns);
   }
   if (!ok || *abort_flag) {
-    // Wind down: let every copy this thread started land before the CTA exits.
+    // Wind down: let every copy this lane started land before the CTA exits.
     volatile int no_abort = 0;
-    for (int s = 0; s < Lay::kNK; ++s) {
-      const int n = kt / Lay::kNK + (s < kt % Lay::kNK ? 1 : 0);
-      if (n > 0) mbar_wait(bars + 8u * (Lay::kBarKFull + s), (n - 1) & 1, &no_abort, 20000000ull);
+    for (int ss = 0; ss < depth; ++ss) {
+      const int nf = n / depth + (ss < n % depth ? 1 : 0);
+      if (nf > 0) mbar_wait(full0 + 8u * ss, (nf - 1) & 1, &no_abort, 20000000ull);
     }
-    for (int s = 0; s < Lay::kNV; ++s) {
-      const int n = vt / Lay::kNV + (s < vt % Lay::kNV ? 1 : 0);
-      if (n > 0) mbar_wait(bars + 8u * (Lay::kBarVFull + s), (n - 1) & 1, &no_abort, 20000000ull);
-    }
-    if (q_issued > 0)
+    if (!is_v && q_issued > 0)
       mbar_wait(bars + 8u * Lay::kBarQFull, (q_issued - 1) & 1, &no_abort, 20000000ull);
   }
 }
@@ -608,7 +602,7 @@ __device__ __forceinline__ void mma_role(const AttnArgs& a, uint8_t* smem, uint3
     }
     if (elect_one()) {
       mma_commit(bars + 8u * (Lay::kBarSFull + kSPerGroup * w + sb));
-      mma_commit(bars + 8u * (Lay::kBarKEmpty + 2 * slot + w));
+      mma_commit(bars + 8u * (Lay::kBarKEmpty + slot));
     }
     __syncwarp();
     return true;
@@ -667,6 +661,9 @@ __device__ __forceinline__ void mma_role(const AttnArgs& a, uint8_t* smem, uint3
       if (qs.t == qs.sg.t0 && !wait(bars + 8u * Lay::kBarQFull, qs.si & 1)) { ok = false; break; }
       bool issued = false;
       if ((qs.it & 1) == w) {
+        // S buffer mq & 1 last held P of own tile mq - 2: its PV must have
+        // finished reading P before this QK overwrites the columns.
+        if (mq >= 2 && !wait(bars + 8u * (Lay::kBarOReady + w), (mq - 2) & 1)) { ok = false; break; }
         if (!issue_qk(qs, mq)) { ok = false; break; }
         ++mq;
         issued = true;
@@ -927,8 +924,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const uint32_t bars = smem_u32(smem) + Lay::kBarOff;
     for (int s = 0; s < Lay::kNK; ++s) {
       mbar_init(bars + 8u * (Lay::kBarKFull + s), 1);
-      mbar_init(bars + 8u * (Lay::kBarKEmpty + 2 * s), 1);
-      mbar_init(bars + 8u * (Lay::kBarKEmpty + 2 * s + 1), 1);
+      mbar_init(bars + 8u * (Lay::kBarKEmpty + s), 1);
     }
     for (int s = 0; s < Lay::kNV; ++s) {
       mbar_init(bars + 8u * (Lay::kBarVFull + s), 1);
@@ -965,7 +961,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == kProducerWarp) {
-    if ((threadIdx.x & 31) == 0)
+    if ((threadIdx.x & 31) < 2)
       producer_role<D>(a, smem, &tm_q, &tm_kc, &tm_vc, &tm_kb, &tm_vb, abort_flag, tab, start);
   } else if (warp < kSoftmaxWarp0) {
     mma_role<D>(a, smem, tmem, abort_flag, warp - kMmaWarp0, tab, start);
