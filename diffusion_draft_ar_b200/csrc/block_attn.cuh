@@ -304,6 +304,8 @@ __device__ __forceinline__ bool schedule_prologue(const AttnArgs& a, uint8_t* sm
 
   long long part = 0;
   for (int b = tid; b < a.B; b += kAttnThreads) {
+    if (blockIdx.x == 0 && (seq_rows_bad(a, b) || seq_len_bad(a, b)))
+      raise_flag(a, ORTHRUS_FLAG_BAD_LENGTH);
     const SeqInfo si = seq_info_global(a, b);
     if (b < kSeqTableCap) rows[b] = make_int4(si.nt, si.L, si.Kb, si.row0);
     part += (long long)a.Hkv * si.nt;
@@ -661,9 +663,6 @@ __device__ __forceinline__ void mma_role(const AttnArgs& a, uint8_t* smem, uint3
       if (qs.t == qs.sg.t0 && !wait(bars + 8u * Lay::kBarQFull, qs.si & 1)) { ok = false; break; }
       bool issued = false;
       if ((qs.it & 1) == w) {
-        // S buffer mq & 1 last held P of own tile mq - 2: its PV must have
-        // finished reading P before this QK overwrites the columns.
-        if (mq >= 2 && !wait(bars + 8u * (Lay::kBarOReady + w), (mq - 2) & 1)) { ok = false; break; }
         if (!issue_qk(qs, mq)) { ok = false; break; }
         ++mq;
         issued = true;
@@ -1000,10 +999,6 @@ __global__ void __launch_bounds__(kCombineRows * 32)
   const int u = blockIdx.x;
   const int b = u / a.Hkv, h = u % a.Hkv;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (u == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
-    for (int bb = 0; bb < a.B; ++bb)
-      if (seq_rows_bad(a, bb) || seq_len_bad(a, bb)) raise_flag(a, ORTHRUS_FLAG_BAD_LENGTH);
-  }
   const int Kb = (b < a.B) ? seq_block_len(a, b) : 0;
   if (Kb <= 0) return;
   const int nt = seq_tiles(a, b);

@@ -102,6 +102,7 @@ bool make_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims
 
 struct AttnPlan {
   int G, R_max, grid, chunked, chunk_tiles, max_chunks, parts;
+  bool combine;  // units may be cut across CTAs: launch the combine kernel
   size_t ws_o_bytes, ws_lse_bytes, ws_bytes;
 };
 
@@ -153,22 +154,33 @@ orthrus_status_t plan_attn(const orthrus_attn_params* p, int sms, AttnPlan* pl) 
     pl->max_chunks = static_cast<int>(mc);
     pl->grid = static_cast<int>(grid);
     pl->parts = pl->grid;
+    pl->combine = true;
+  } else if (p->max_ctas == 0 && static_cast<long long>(p->B) * p->Hkv >= (3LL * sms) / 4 &&
+             static_cast<long long>(p->B) * p->Hkv <= sms) {
+    // When the (sequence, KV head) units number between 3/4 of the SMs and
+    // the SM count, one CTA per whole unit leaves a few SMs idle but cuts no
+    // unit: no partials, no combine launch, and no unit switch inside a CTA
+    // (each switch drains the pipeline while the next unit's Q tile loads).
+    // This is the fixed-chunk schedule with one chunk per unit. A batch whose
+    // prefix lengths differ widely is better served by max_ctas = SM count.
+    const long long ptiles = (max_tokens + kTileN - 1) / kTileN;
+    pl->chunked = 1;
+    pl->chunk_tiles = static_cast<int>(ptiles > 0 ? ptiles : 1);
+    pl->max_chunks = 1;
+    pl->grid = p->B * p->Hkv;
+    pl->parts = pl->grid;
+    pl->combine = false;
   } else {
     pl->chunked = 0;
     pl->chunk_tiles = 0;
     pl->max_chunks = 0;
-    // Balanced ranges over one CTA per SM. When the (sequence, KV head) units
-    // number between 3/4 of the SMs and the SM count, one CTA per unit leaves
-    // a few SMs idle but cuts no unit, which saves the partial/merge work and
-    // the in-CTA unit switches that a near-one-unit range split would add.
-    const long long units = static_cast<long long>(p->B) * p->Hkv;
-    int auto_ctas = sms;
-    if (units >= (3LL * sms) / 4 && units <= sms) auto_ctas = static_cast<int>(units);
-    int c = p->max_ctas > 0 ? p->max_ctas : auto_ctas;
+    // Balanced ranges over one CTA per SM (or max_ctas).
+    int c = p->max_ctas > 0 ? p->max_ctas : sms;
     if (c < 1) c = 1;
     if (c > 65535) c = 65535;
     pl->grid = c;
     pl->parts = 2 * c;
+    pl->combine = true;
   }
   pl->ws_o_bytes = round_up(static_cast<size_t>(pl->parts) * kTileM * p->D * sizeof(float), 256);
   pl->ws_lse_bytes = round_up(static_cast<size_t>(pl->parts) * kTileM * sizeof(float), 256);
@@ -253,6 +265,7 @@ orthrus_status_t launch_attn(const orthrus_attn_params* p, const AttnPlan& pl, i
   block_attn_kernel<D><<<pl.grid, kAttnThreads, Lay::kAlloc, stream>>>(tq, tkc, tvc, tkb, tvb, a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return fail(ORTHRUS_ERR_CUDA, "block_attn launch: %s", cudaGetErrorString(e));
+  if (!pl.combine) return ok();
   // The combine kernel is launched as a programmatic dependent of the
   // attention grid: its launch and schedule prologue overlap the attention
   // tail, and it reads the partials only after griddepcontrol.wait.

@@ -115,7 +115,10 @@ typedef struct {
   float softmax_scale;       /* <= 0: 1/sqrt(D) */
   int32_t kv_split_tokens;   /* 0: balanced split over the SMs; > 0: fixed chunks of this
                                 many prefix tokens (a multiple of 64), one CTA each */
-  int32_t max_ctas;          /* 0: one CTA per SM; > 0: cap for the balanced split */
+  int32_t max_ctas;          /* 0: library picks: one CTA per (sequence, KV head) unit
+                                when the units number between 3/4 of the SM count and
+                                the SM count, else a balanced split over one CTA per SM;
+                                > 0: balanced split over this many CTAs */
   void* out;                 /* device bf16 [R, Hq, D] */
   void* workspace;           /* device scratch, >= orthrus_block_attn_workspace_size() bytes,
                                 256-byte aligned; contents need no initialisation */
