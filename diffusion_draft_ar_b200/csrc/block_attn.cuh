@@ -64,7 +64,7 @@ struct AttnArgs {
   const int* cu_block;
   const int* page_table;
   __nv_bfloat16* out;
-  float* ws_o;     // partial accumulators [parts][128][D]
+  float* ws_o;     // partial accumulators [parts][4 row blocks][D][32 rows] (see part_o)
   float* ws_lse;   // partial log2-sum-exp  [parts][128]
   int* error_flag;
   float scale_log2;  // softmax scale * log2(e)
@@ -76,6 +76,7 @@ struct AttnArgs {
   int num_ctas;      // grid size
   unsigned long long timeout_ns;
   int fault_inject;  // test hook: 1 drops each CTA's first V copy (a wait must time out)
+  int out_v8;        // out is 32-byte aligned: rows are written with 256-bit stores
 };
 
 // ---------------------------------------------------------------------------
@@ -265,6 +266,15 @@ __device__ __forceinline__ int tile_valid_keys(int t, int L, int np, int Kb) {
   if (t == np) return Kb;
   const int rem = L - t * kTileN;
   return rem < kTileN ? rem : kTileN;
+}
+
+// Partial accumulator of query row r (0..127), column c, in part p. Each warp
+// of a softmax group holds 32 consecutive rows (one TMEM lane quarter), so
+// the layout keeps those 32 rows contiguous per column: one warp-wide store
+// of a column writes 128 contiguous bytes, and the combine reads the same way.
+template <int D>
+__device__ __forceinline__ long long part_o(int p, int r, int c) {
+  return ((long long)p * kTileM + (r >> 5) * 32) * D + (long long)c * 32 + (r & 31);
 }
 
 __device__ __forceinline__ void raise_flag(const AttnArgs& a, int bits) {
@@ -649,7 +659,11 @@ __device__ __forceinline__ void mma_role(const AttnArgs& a, uint8_t* smem, uint3
     return true;
   };
 
-  // QK walk over every tile: Q waits and commits at segment edges, QK for own tiles.
+  // QK walk over every tile: Q waits and commits at segment edges, QK for own
+  // tiles, up to two own tiles ahead of PV. The walk holds at the end of a
+  // unit while PVs of that unit are still to be issued: they go first, so the
+  // unit's last PVs (and the epilogue waiting on them) never queue behind the
+  // next unit's QKs, which must wait for that unit's Q tile to load.
   TileStep qs;
   qs.cur = start;
   qs.si = -1;
@@ -657,23 +671,34 @@ __device__ __forceinline__ void mma_role(const AttnArgs& a, uint8_t* smem, uint3
   qs.valid = false;
   TileStep ps = qs;
   int mq = 0, mp = 0;  // own tiles issued (QK) / (PV)
-  bool ok = true;
-  auto advance_qk = [&]() -> bool {  // issue the next own QK; false at the end
-    while (ok && step_next(a, tab, qs)) {
-      if (qs.t == qs.sg.t0 && !wait(bars + 8u * Lay::kBarQFull, qs.si & 1)) { ok = false; break; }
-      bool issued = false;
+  bool ok = true, qk_pending = false, qk_done = false;
+  auto commit_q_empty = [&]() {
+    if (elect_one()) mma_commit(bars + 8u * Lay::kBarQEmpty);
+    __syncwarp();
+  };
+  auto walk_qk = [&]() {  // move qs to the next own tile
+    while (ok) {
+      if (qs.valid && qs.t + 1 >= qs.sg.t1 && mp < mq) return;  // hold at the unit's end
+      if (!step_next(a, tab, qs)) {
+        qk_done = true;
+        return;
+      }
+      if (qs.t == qs.sg.t0 && !wait(bars + 8u * Lay::kBarQFull, qs.si & 1)) { ok = false; return; }
       if ((qs.it & 1) == w) {
-        if (!issue_qk(qs, mq)) { ok = false; break; }
-        ++mq;
-        issued = true;
+        qk_pending = true;
+        return;
       }
-      if (qs.t == qs.sg.t1 - 1) {
-        if (elect_one()) mma_commit(bars + 8u * Lay::kBarQEmpty);
-        __syncwarp();
-      }
-      if (issued) return true;
+      if (qs.t == qs.sg.t1 - 1) commit_q_empty();
     }
-    return false;
+  };
+  auto try_qk = [&]() -> bool {  // issue the next own QK unless held
+    if (!qk_pending && !qk_done) walk_qk();
+    if (!ok || !qk_pending) return false;
+    if (!issue_qk(qs, mq)) { ok = false; return false; }
+    ++mq;
+    qk_pending = false;
+    if (qs.t == qs.sg.t1 - 1) commit_q_empty();
+    return true;
   };
   auto advance_pv = [&]() -> bool {
     while (ok && step_next(a, tab, ps)) {
@@ -686,10 +711,11 @@ __device__ __forceinline__ void mma_role(const AttnArgs& a, uint8_t* smem, uint3
     }
     return false;
   };
-  advance_qk();
-  advance_qk();
-  while (ok && advance_pv()) advance_qk();
-  while (ok && advance_qk()) {}  // finish the Q bookkeeping walk
+  while (ok) {
+    while (ok && mq - mp < 2 && try_qk()) {}
+    if (!ok || mp == mq) break;  // every QK issued (walk done) and every PV too
+    if (!advance_pv()) break;
+  }
   // Drain: every MMA issued above completes before TMEM is released.
   if (elect_one()) {
     mma_commit(bars + 8u * (Lay::kBarDrain + w));
@@ -873,17 +899,30 @@ __device__ __forceinline__ void softmax_role(const AttnArgs& a, uint8_t* smem, u
       if (my_valid) {
         if (sg.part < 0) {
           __nv_bfloat16* dst = a.out + ((long long)(row0 + irow) * a.Hq + h * a.G + g) * D + col;
-          uint4* d4 = reinterpret_cast<uint4*>(dst);
+          if (a.out_v8) {
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            d4[k] = make_uint4(pack_bf16x2(o[8 * k + 0], o[8 * k + 1]),
-                               pack_bf16x2(o[8 * k + 2], o[8 * k + 3]),
-                               pack_bf16x2(o[8 * k + 4], o[8 * k + 5]),
-                               pack_bf16x2(o[8 * k + 6], o[8 * k + 7]));
+            for (int k = 0; k < 2; ++k)
+              st_global_v8(dst + 16 * k, pack_bf16x2(o[16 * k + 0], o[16 * k + 1]),
+                           pack_bf16x2(o[16 * k + 2], o[16 * k + 3]),
+                           pack_bf16x2(o[16 * k + 4], o[16 * k + 5]),
+                           pack_bf16x2(o[16 * k + 6], o[16 * k + 7]),
+                           pack_bf16x2(o[16 * k + 8], o[16 * k + 9]),
+                           pack_bf16x2(o[16 * k + 10], o[16 * k + 11]),
+                           pack_bf16x2(o[16 * k + 12], o[16 * k + 13]),
+                           pack_bf16x2(o[16 * k + 14], o[16 * k + 15]));
+          } else {
+            uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              d4[k] = make_uint4(pack_bf16x2(o[8 * k + 0], o[8 * k + 1]),
+                                 pack_bf16x2(o[8 * k + 2], o[8 * k + 3]),
+                                 pack_bf16x2(o[8 * k + 4], o[8 * k + 5]),
+                                 pack_bf16x2(o[8 * k + 6], o[8 * k + 7]));
+          }
         } else {
-          float4* d4 = reinterpret_cast<float4*>(a.ws_o + ((long long)sg.part * kTileM + row) * D + col);
+          float* dst = a.ws_o + part_o<D>(sg.part, row, col);
 #pragma unroll
-          for (int k = 0; k < 8; ++k) d4[k] = make_float4(o[4 * k], o[4 * k + 1], o[4 * k + 2], o[4 * k + 3]);
+          for (int k = 0; k < 32; ++k) dst[32 * k] = o[k];
         }
       }
     }
@@ -977,11 +1016,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
 // ---------------------------------------------------------------------------
 // Combine: merge the partials of every unit that was cut across CTAs.
-// grid = (B * Hkv, ceil(G * max_block / kCombineRows)); one warp per query row.
-// Warp 0 finds the unit's partials once per CTA; the partials themselves are
-// read only after the attention grid's writes are visible (griddepcontrol.wait).
+// grid = (B * Hkv, 4 row blocks of 32 query rows); 4 warps per CTA, lane =
+// query row, warp = a quarter of the D columns. Warp 0 finds the unit's
+// partials once per CTA; the partials themselves are read only after the
+// attention grid's writes are visible (griddepcontrol.wait). The merged rows
+// are staged in shared memory and written out row by row.
 
-constexpr int kCombineRows = 8;
+constexpr int kCombineThreads = 128;
 
 __device__ __forceinline__ int cta_of_tile(long long T, int C, long long t) {
   long long c = ((t + 1) * C - 1) / T;
@@ -992,18 +1033,20 @@ __device__ __forceinline__ int cta_of_tile(long long T, int C, long long t) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(kCombineRows * 32)
+__global__ void __launch_bounds__(kCombineThreads)
     attn_combine_kernel(const AttnArgs a) {
   __shared__ long long sh_T, sh_su;
-  __shared__ int sh_clo, sh_chi, sh_count, sh_skip;
-  const int u = blockIdx.x;
+  __shared__ int sh_clo, sh_count, sh_skip;
+  __shared__ __align__(16) __nv_bfloat16 tile[32][D + 8];
+  const int u = blockIdx.x, rb = blockIdx.y;
   const int b = u / a.Hkv, h = u % a.Hkv;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int Kb = (b < a.B) ? seq_block_len(a, b) : 0;
-  if (Kb <= 0) return;
+  const int rows_valid = a.G * Kb;
+  if (Kb <= 0 || rb * 32 >= rows_valid) return;
   const int nt = seq_tiles(a, b);
   if (warp == 0) {
-    int skip = 0, count = 0, c_lo = 0, c_hi = -1;
+    int skip = 0, count = 0, c_lo = 0;
     long long T = 0, s_u = 0;
     if (a.chunked) {
       count = unit_chunks(a, nt);
@@ -1024,7 +1067,7 @@ __global__ void __launch_bounds__(kCombineRows * 32)
       T = t_part;
       s_u = s_part + (long long)h * nt;
       c_lo = cta_of_tile(T, a.num_ctas, s_u);
-      c_hi = cta_of_tile(T, a.num_ctas, s_u + nt - 1);
+      const int c_hi = cta_of_tile(T, a.num_ctas, s_u + nt - 1);
       skip = c_lo == c_hi;
       count = c_hi - c_lo + 1;
     }
@@ -1032,18 +1075,15 @@ __global__ void __launch_bounds__(kCombineRows * 32)
       sh_T = T;
       sh_su = s_u;
       sh_clo = c_lo;
-      sh_chi = c_hi;
       sh_count = count;
       sh_skip = skip;
     }
   }
   __syncthreads();
   if (sh_skip) return;
-  const int r = blockIdx.y * kCombineRows + warp;
-  if (r >= a.G * Kb) return;
   const long long T = sh_T, s_u = sh_su;
   const int c_lo = sh_clo, count = sh_count;
-  constexpr int kPer = D / 32;  // elements per thread
+  constexpr int kCols = D / 4;  // columns per warp
 
   auto part_of = [&](int k, bool& use) -> int {
     if (a.chunked) {
@@ -1058,15 +1098,16 @@ __global__ void __launch_bounds__(kCombineRows * 32)
   };
 
   pdl_wait();  // partials written by the attention grid are visible from here on
+  const int r = rb * 32 + lane;  // query row of this lane (rows past rows_valid are ignored)
   float M = -__int_as_float(0x7f800000);
   for (int k = 0; k < count; ++k) {
     bool use;
     const int p = part_of(k, use);
     if (use) M = fmaxf(M, a.ws_lse[(long long)p * kTileM + r]);
   }
-  float acc[kPer];
+  float acc[kCols];
 #pragma unroll
-  for (int e = 0; e < kPer; ++e) acc[e] = 0.f;
+  for (int e = 0; e < kCols; ++e) acc[e] = 0.f;
   float wsum = 0.f;
   for (int k = 0; k < count; ++k) {
     bool use;
@@ -1074,21 +1115,27 @@ __global__ void __launch_bounds__(kCombineRows * 32)
     if (!use) continue;
     const float wgt = exp2f(a.ws_lse[(long long)p * kTileM + r] - M);
     wsum += wgt;
-    const float* src = a.ws_o + ((long long)p * kTileM + r) * D + lane * kPer;
+    const float* src = a.ws_o + part_o<D>(p, r, warp * kCols);
 #pragma unroll
-    for (int e = 0; e < kPer; e += 2) {
-      const float2 x = *reinterpret_cast<const float2*>(src + e);
-      acc[e] = fmaf(wgt, x.x, acc[e]);
-      acc[e + 1] = fmaf(wgt, x.y, acc[e + 1]);
-    }
+    for (int e = 0; e < kCols; ++e) acc[e] = fmaf(wgt, src[32 * e], acc[e]);
   }
   const float inv = 1.f / wsum;
-  const int i = r / a.G, g = r - i * a.G;
-  __nv_bfloat16* dst =
-      a.out + ((long long)(seq_row0(a, b) + i) * a.Hq + h * a.G + g) * D + lane * kPer;
 #pragma unroll
-  for (int e = 0; e < kPer; e += 2)
-    *reinterpret_cast<uint32_t*>(dst + e) = pack_bf16x2(acc[e] * inv, acc[e + 1] * inv);
+  for (int e = 0; e < kCols; e += 2)
+    *reinterpret_cast<uint32_t*>(&tile[lane][warp * kCols + e]) =
+        pack_bf16x2(acc[e] * inv, acc[e + 1] * inv);
+  __syncthreads();
+  // each query row is D contiguous bf16 in out; 16-byte pieces, row-major
+  const int row0 = seq_row0(a, b);
+  constexpr int kPieces = D / 8;
+  for (int idx = tid; idx < 32 * kPieces; idx += kCombineThreads) {
+    const int rr = idx / kPieces, pc = idx % kPieces;
+    const int q = rb * 32 + rr;
+    if (q >= rows_valid) continue;
+    const int i = q / a.G, g = q - i * a.G;
+    __nv_bfloat16* dst = a.out + ((long long)(row0 + i) * a.Hq + h * a.G + g) * D + pc * 8;
+    *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(&tile[rr][pc * 8]);
+  }
 }
 
 }  // namespace orthrus

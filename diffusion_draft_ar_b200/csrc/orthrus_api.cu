@@ -261,6 +261,7 @@ orthrus_status_t launch_attn(const orthrus_attn_params* p, const AttnPlan& pl, i
     const char* fi = std::getenv("ORTHRUS_FAULT_INJECT");
     a.fault_inject = fi ? std::atoi(fi) : 0;
   }
+  a.out_v8 = aligned(p->out, 32) ? 1 : 0;
 
   block_attn_kernel<D><<<pl.grid, kAttnThreads, Lay::kAlloc, stream>>>(tq, tkc, tvc, tkb, tvb, a);
   cudaError_t e = cudaGetLastError();
@@ -269,10 +270,10 @@ orthrus_status_t launch_attn(const orthrus_attn_params* p, const AttnPlan& pl, i
   // The combine kernel is launched as a programmatic dependent of the
   // attention grid: its launch and schedule prologue overlap the attention
   // tail, and it reads the partials only after griddepcontrol.wait.
-  const int row_groups = (pl.G * p->max_block + kCombineRows - 1) / kCombineRows;
+  const int row_blocks = (pl.G * p->max_block + 31) / 32;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(p->B * p->Hkv, row_groups);
-  cfg.blockDim = dim3(kCombineRows * 32);
+  cfg.gridDim = dim3(p->B * p->Hkv, row_blocks);
+  cfg.blockDim = dim3(kCombineThreads);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
