@@ -216,8 +216,8 @@ struct AttnLayout {
   static constexpr int kBarQFull = kBarVEmpty + kNV;
   static constexpr int kBarQEmpty = kBarQFull + 1;
   static constexpr int kBarSFull = kBarQEmpty + 1;             // [2 groups][kSPerGroup]
-  static constexpr int kBarPReady = kBarSFull + 2 * kSPerGroup;  // [2]
-  static constexpr int kBarOReady = kBarPReady + 2;      // [2]
+  static constexpr int kBarPReady = kBarSFull + 2 * kSPerGroup;  // [2 groups][2]
+  static constexpr int kBarOReady = kBarPReady + 4;      // [2]
   static constexpr int kBarOFree = kBarOReady + 2;
   static constexpr int kBarXchg = kBarOFree + 1;
   static constexpr int kBarDrain = kBarXchg + 1;  // [2]
@@ -624,7 +624,7 @@ __device__ __forceinline__ void mma_role(const AttnArgs& a, uint8_t* smem, uint3
     const int slot = j.it % Lay::kNV;
     // p_ready also means the tile's V copy has landed: the softmax group waits
     // for it before publishing P, which keeps that wait off this warp's path.
-    if (!wait(bars + 8u * (Lay::kBarPReady + w), m & 1)) return false;
+    if (!wait(bars + 8u * (Lay::kBarPReady + 2 * w + (m & 1)), (m >> 1) & 1)) return false;
     const int nvalid = tile_valid_keys(j.t, j.L, j.np, j.Kb);
     if (nvalid < kTileN) {
       // Rows past the last valid key may hold stale or non-finite data;
@@ -800,13 +800,27 @@ __device__ __forceinline__ void softmax_role(const AttnArgs& a, uint8_t* smem, u
       const float m_new = fmaxf(m_ref, mt * c);
       const bool need = has && (m_new > m_ref + kRescaleLog2);
       if (!has) m_ref = m_new;
-      // The previous PV of this group must be done before O is rescaled (and
-      // the wait keeps this group's o_ready phases in step).
-      if (cnt > 0 && pv_waited < cnt) {
+      // S of own tile cnt is complete, so are the PVs of own tiles 0 .. cnt-2:
+      // the MMA warp issued them before this QK, and one thread's tcgen05
+      // operations complete in order. Only the PV of own tile cnt-1 may still
+      // run. It is waited for only when O must be rescaled (so this tile's
+      // exponentials overlap it) and at the group's last tile of the unit
+      // (so at most one PV is pending at the unit's end). Each o_ready wait
+      // is for the oldest unobserved phase with at most one phase in flight,
+      // so the parity is exact. P_ready alternates between two barriers per
+      // group, so P of tile cnt may be published before the MMA warp has
+      // taken P of tile cnt-1.
+      if (pv_waited < cnt - 1) pv_waited = cnt - 1;
+      const bool unit_last = t + 2 >= sg.t1;
+      if (unit_last && pv_waited < cnt) {
         if (!wait(bar(Lay::kBarOReady + w), pv_waited & 1)) { ok = false; break; }
         ++pv_waited;
       }
       if (__any_sync(0xffffffffu, need)) {
+        if (pv_waited < cnt) {
+          if (!wait(bar(Lay::kBarOReady + w), pv_waited & 1)) { ok = false; break; }
+          ++pv_waited;
+        }
         const float alpha = need ? ex2_approx(m_ref - m_new) : 1.f;
         if (need) {
           l_sum *= alpha;
@@ -847,7 +861,7 @@ __device__ __forceinline__ void softmax_role(const AttnArgs& a, uint8_t* smem, u
       has = true;
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar(Lay::kBarPReady + w));
+      mbar_arrive(bar(Lay::kBarPReady + 2 * w + (cnt & 1)));
       ++cnt;
     }
     if (!ok) break;
@@ -972,7 +986,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     mbar_init(bars + 8u * Lay::kBarQEmpty, 2);  // one arrival per MMA warp
     for (int k = 0; k < 2 * kSPerGroup; ++k) mbar_init(bars + 8u * (Lay::kBarSFull + k), 1);
     for (int w = 0; w < 2; ++w) {
-      mbar_init(bars + 8u * (Lay::kBarPReady + w), 128);
+      mbar_init(bars + 8u * (Lay::kBarPReady + 2 * w), 128);
+      mbar_init(bars + 8u * (Lay::kBarPReady + 2 * w + 1), 128);
       mbar_init(bars + 8u * (Lay::kBarOReady + w), 1);
     }
     mbar_init(bars + 8u * Lay::kBarOFree, 256);
