@@ -1031,13 +1031,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
 // ---------------------------------------------------------------------------
 // Combine: merge the partials of every unit that was cut across CTAs.
-// grid = (B * Hkv, 4 row blocks of 32 query rows); 4 warps per CTA, lane =
-// query row, warp = a quarter of the D columns. Warp 0 finds the unit's
-// partials once per CTA; the partials themselves are read only after the
-// attention grid's writes are visible (griddepcontrol.wait). The merged rows
-// are staged in shared memory and written out row by row.
+// grid = (B * Hkv, 4 blocks of 32 query rows, 1 or D / 32); 8 warps per CTA,
+// lane = query row. With a third grid dimension of D / 32 (fixed chunks: many
+// partials per unit) each CTA owns 32 columns and its 8 warps split the
+// partials; with 1 (balanced split: two or three partials) the warps split
+// the column blocks and, within each, the partials. Warp 0 finds the unit's partials once per CTA; the
+// partials themselves are read only after the attention grid's writes are
+// visible (griddepcontrol.wait).
 
-constexpr int kCombineThreads = 128;
+constexpr int kCombineWarps = 8;
+constexpr int kCombineThreads = 32 * kCombineWarps;
 
 __device__ __forceinline__ int cta_of_tile(long long T, int C, long long t) {
   long long c = ((t + 1) * C - 1) / T;
@@ -1052,7 +1055,9 @@ __global__ void __launch_bounds__(kCombineThreads)
     attn_combine_kernel(const AttnArgs a) {
   __shared__ long long sh_T, sh_su;
   __shared__ int sh_clo, sh_count, sh_skip;
-  __shared__ __align__(16) __nv_bfloat16 tile[32][D + 8];
+  __shared__ float sh_m[kCombineWarps][32];
+  __shared__ float sh_w[kCombineWarps][32];
+  __shared__ float sh_acc[kCombineWarps][32][33];
   const int u = blockIdx.x, rb = blockIdx.y;
   const int b = u / a.Hkv, h = u % a.Hkv;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -1098,7 +1103,6 @@ __global__ void __launch_bounds__(kCombineThreads)
   if (sh_skip) return;
   const long long T = sh_T, s_u = sh_su;
   const int c_lo = sh_clo, count = sh_count;
-  constexpr int kCols = D / 4;  // columns per warp
 
   auto part_of = [&](int k, bool& use) -> int {
     if (a.chunked) {
@@ -1114,42 +1118,61 @@ __global__ void __launch_bounds__(kCombineThreads)
 
   pdl_wait();  // partials written by the attention grid are visible from here on
   const int r = rb * 32 + lane;  // query row of this lane (rows past rows_valid are ignored)
-  float M = -__int_as_float(0x7f800000);
-  for (int k = 0; k < count; ++k) {
+  const float NEG_INF = -__int_as_float(0x7f800000);
+  // 1. the row's maximum log-sum-exp over all partials
+  float M = NEG_INF;
+  for (int k = warp; k < count; k += kCombineWarps) {
     bool use;
     const int p = part_of(k, use);
     if (use) M = fmaxf(M, a.ws_lse[(long long)p * kTileM + r]);
   }
-  float acc[kCols];
+  sh_m[warp][lane] = M;
+  __syncthreads();
 #pragma unroll
-  for (int e = 0; e < kCols; ++e) acc[e] = 0.f;
+  for (int k = 0; k < kCombineWarps; ++k) M = fmaxf(M, sh_m[k][lane]);
+  // 2. warps split over (column block, partial class): the CTA covers
+  // ncb = (D / 32) / gridDim.z column blocks, wpc = 8 / ncb warps per block;
+  // warp w takes column block blockIdx.z + (w / wpc) * gridDim.z and the
+  // partials k = w % wpc, w % wpc + wpc, ...
+  const int ncb = (D / 32) / gridDim.z;
+  const int wpc = kCombineWarps / ncb;
+  const int cb = blockIdx.z + (warp / wpc) * gridDim.z;
+  const int kw = warp % wpc;
+  float acc[32];
+#pragma unroll
+  for (int e = 0; e < 32; ++e) acc[e] = 0.f;
   float wsum = 0.f;
-  for (int k = 0; k < count; ++k) {
+  for (int k = kw; k < count; k += wpc) {
     bool use;
     const int p = part_of(k, use);
     if (!use) continue;
     const float wgt = exp2f(a.ws_lse[(long long)p * kTileM + r] - M);
     wsum += wgt;
-    const float* src = a.ws_o + part_o<D>(p, r, warp * kCols);
+    const float* src = a.ws_o + part_o<D>(p, r, cb * 32);
 #pragma unroll
-    for (int e = 0; e < kCols; ++e) acc[e] = fmaf(wgt, src[32 * e], acc[e]);
+    for (int e = 0; e < 32; ++e) acc[e] = fmaf(wgt, src[32 * e], acc[e]);
   }
-  const float inv = 1.f / wsum;
+  sh_w[warp][lane] = wsum;
 #pragma unroll
-  for (int e = 0; e < kCols; e += 2)
-    *reinterpret_cast<uint32_t*>(&tile[lane][warp * kCols + e]) =
-        pack_bf16x2(acc[e] * inv, acc[e + 1] * inv);
+  for (int e = 0; e < 32; ++e) sh_acc[warp][lane][e] = acc[e];
   __syncthreads();
-  // each query row is D contiguous bf16 in out; 16-byte pieces, row-major
+  // 3. reduce each column block's wpc warps: thread -> (block, row, column pair)
   const int row0 = seq_row0(a, b);
-  constexpr int kPieces = D / 8;
-  for (int idx = tid; idx < 32 * kPieces; idx += kCombineThreads) {
-    const int rr = idx / kPieces, pc = idx % kPieces;
+  for (int idx = tid; idx < ncb * 32 * 16; idx += kCombineThreads) {
+    const int j = idx / (32 * 16), rr = (idx >> 4) & 31, e = (idx & 15) * 2;
     const int q = rb * 32 + rr;
     if (q >= rows_valid) continue;
+    float w = 0.f, x0 = 0.f, x1 = 0.f;
+    for (int k = j * wpc; k < (j + 1) * wpc; ++k) {
+      w += sh_w[k][rr];
+      x0 += sh_acc[k][rr][e];
+      x1 += sh_acc[k][rr][e + 1];
+    }
+    const float inv = 1.f / w;
     const int i = q / a.G, g = q - i * a.G;
-    __nv_bfloat16* dst = a.out + ((long long)(row0 + i) * a.Hq + h * a.G + g) * D + pc * 8;
-    *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(&tile[rr][pc * 8]);
+    const int c = (blockIdx.z + j * gridDim.z) * 32 + e;
+    __nv_bfloat16* dst = a.out + ((long long)(row0 + i) * a.Hq + h * a.G + g) * D + c;
+    *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(x0 * inv, x1 * inv);
   }
 }
 

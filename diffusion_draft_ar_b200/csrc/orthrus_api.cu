@@ -272,7 +272,10 @@ orthrus_status_t launch_attn(const orthrus_attn_params* p, const AttnPlan& pl, i
   // tail, and it reads the partials only after griddepcontrol.wait.
   const int row_blocks = (pl.G * p->max_block + 31) / 32;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(p->B * p->Hkv, row_blocks);
+  // Fixed chunks leave many partials per unit: spread a row block's columns
+  // over D / 32 CTAs. A balanced split leaves two or three: one CTA per row
+  // block is enough.
+  cfg.gridDim = dim3(p->B * p->Hkv, row_blocks, pl.chunked ? D / 32 : 1);
   cfg.blockDim = dim3(kCombineThreads);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = stream;
