@@ -290,6 +290,9 @@ def run_ours(args):
         params[view] = p
     for p in params.values():
         p.workspace, p.workspace_bytes = ws_attn.data_ptr(), ws_attn.numel()
+    # our kernels per step: both attention calls (1 or 2 kernels each),
+    # consensus (argmax + finalize) and kv_append
+    launches_per_step = sum(O.block_attn_kernel_count(p) for p in params.values()) + 2 + 1
     targets = torch.argmax(r.logits, dim=1).to(torch.int32)
     drafts = wi.drafts(0, targets)
     acc = torch.zeros(m.B, dtype=torch.int32, device=dev)
@@ -433,7 +436,7 @@ def run_ours(args):
                     "note": "per step: pinned H2D of both views' q/k/v blocks, logits and drafts; "
                             "D2H of both outputs, accept lengths and next tokens; "
                             "the KV cache stays resident"},
-            "gpu_launches": args.steps * 7,
+            "gpu_launches": args.steps * launches_per_step,
             "clocks": clocks,
         }
         print(json.dumps(line), flush=True)

@@ -302,6 +302,15 @@ size_t orthrus_block_attn_workspace_size(const orthrus_attn_params* p) {
   return pl.ws_bytes;
 }
 
+int32_t orthrus_block_attn_kernel_count(const orthrus_attn_params* p) {
+  int sms = 0;
+  if (!p) return 0;
+  if (p->kv_split_tokens == 0 && p->max_ctas == 0 && device_sm_count(&sms) < 0) return 0;
+  AttnPlan pl;
+  if (plan_attn(p, sms, &pl) != ORTHRUS_OK) return 0;
+  return pl.combine ? 2 : 1;
+}
+
 orthrus_status_t orthrus_block_attn(const orthrus_attn_params* p, void* stream) {
   AttnPlan pl;
   orthrus_status_t s = plan_attn(p, 1, &pl);  // geometry checks first, no CUDA call

@@ -48,6 +48,8 @@ class AttnParams(ctypes.Structure):
 
 lib.orthrus_block_attn_workspace_size.restype = _sz
 lib.orthrus_block_attn_workspace_size.argtypes = [ctypes.POINTER(AttnParams)]
+lib.orthrus_block_attn_kernel_count.restype = _i32
+lib.orthrus_block_attn_kernel_count.argtypes = [ctypes.POINTER(AttnParams)]
 lib.orthrus_block_attn.restype = _i32
 lib.orthrus_block_attn.argtypes = [ctypes.POINTER(AttnParams), _vp]
 lib.orthrus_consensus_workspace_size.restype = _sz
@@ -138,6 +140,11 @@ def attn_params(view, q_block, k_cache, v_cache, k_block, v_block, prefix_lens, 
 
 def block_attn_workspace_size(params: AttnParams) -> int:
     return int(lib.orthrus_block_attn_workspace_size(ctypes.byref(params)))
+
+
+def block_attn_kernel_count(params: AttnParams) -> int:
+    """Kernels one ``orthrus_block_attn`` call with these parameters launches."""
+    return int(lib.orthrus_block_attn_kernel_count(ctypes.byref(params)))
 
 
 def block_attn(view, q_block, k_cache, v_cache, k_block, v_block, prefix_lens, cu_block,

@@ -130,6 +130,13 @@ typedef struct {
  * current device's SM count). 0 when the parameters are invalid. */
 ORTHRUS_API size_t orthrus_block_attn_workspace_size(const orthrus_attn_params* p);
 
+/* Number of kernels one orthrus_block_attn call with these parameters launches
+ * on the current device: 1 when no (sequence, KV head) unit is cut across CTAs
+ * (one CTA per whole unit, chosen when the units number between 3/4 of the SM
+ * count and the SM count), 2 otherwise (attention, then the combine kernel
+ * that merges the partials). 0 when the parameters are invalid. */
+ORTHRUS_API int32_t orthrus_block_attn_kernel_count(const orthrus_attn_params* p);
+
 /* Launch the block attention described by *p on `stream`.
  * q_block, k_block, v_block and out hold total_rows rows; a sequence whose
  * cu_block range is decreasing, longer than max_block or past total_rows is

@@ -113,6 +113,16 @@ def test_block_attn_workspace_size_chunked_mode(O):
     assert O.block_attn_workspace_size(_params(O, D=96, kv_split_tokens=64)) == 0
 
 
+def test_block_attn_kernel_count(O):
+    # fixed chunks and an explicit CTA cap always merge partials: two kernels;
+    # invalid parameters: 0 (both decided on the host, no device query)
+    p = _params(O, B=1, Hq=32, Hkv=8, max_block=32, total_rows=32, max_pages_per_seq=2049,
+                num_pages=2049, kv_split_tokens=2048)
+    assert O.block_attn_kernel_count(p) == 2
+    assert O.block_attn_kernel_count(_params(O, max_ctas=7)) == 2
+    assert O.block_attn_kernel_count(_params(O, D=96, kv_split_tokens=64)) == 0
+
+
 @pytest.mark.parametrize("args,status", [
     (dict(V=0), 1), (dict(ld=10, V=20), 1), (dict(B=-1), 1), (dict(max_block=0), 1),
     (dict(logits=None), 1), (dict(draft=None), 1), (dict(workspace=None), 1),
