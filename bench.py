@@ -291,8 +291,10 @@ def run_ours(args):
     for p in params.values():
         p.workspace, p.workspace_bytes = ws_attn.data_ptr(), ws_attn.numel()
     # our kernels per step: both attention calls (1 or 2 kernels each),
-    # consensus (argmax + finalize) and kv_append
-    launches_per_step = sum(O.block_attn_kernel_count(p) for p in params.values()) + 2 + 1
+    # consensus (argmax + finalize) and, when the commit is a separate append, kv_append
+    write = args.commit == "write"
+    launches_per_step = (sum(O.block_attn_kernel_count(p) for p in params.values()) + 2 +
+                         (0 if write else 1))
     targets = torch.argmax(r.logits, dim=1).to(torch.int32)
     drafts = wi.drafts(0, targets)
     acc = torch.zeros(m.B, dtype=torch.int32, device=dev)
@@ -305,6 +307,7 @@ def run_ours(args):
     cons_args = (r.logits.data_ptr(), w.vocab, w.vocab, drafts.data_ptr(), cu.data_ptr(), m.B,
                  w.max_block, acc.data_ptr(), nxt.data_ptr(), None, ws_cons.data_ptr(),
                  ws_cons.numel(), sp)
+    commit_args = cons_args[:10] + (lens.data_ptr(),) + cons_args[10:]
     kb, vb = r.k_block["verify"], r.v_block["verify"]
     app_args = (kb.data_ptr(), vb.data_ptr(), cu.data_ptr(), w.max_block, acc.data_ptr(),
                 lens.data_ptr(), 1, table.data_ptr(), m.max_pages, m.num_pages,
@@ -318,13 +321,19 @@ def run_ours(args):
         s1 = L.orthrus_block_attn(P_diff, sp)
         if ev is not None:
             ev[1].record(stream)
-        s2 = L.orthrus_block_attn(P_ver, sp)
+        if write:  # write-then-truncate: VERIFY stores the block K/V, consensus commits
+            s2 = L.orthrus_block_attn_verify_write(P_ver, sp)
+        else:
+            s2 = L.orthrus_block_attn(P_ver, sp)
         if ev is not None:
             ev[2].record(stream)
-        s3 = L.orthrus_consensus(*cons_args)
+        if write:
+            s3 = L.orthrus_consensus_commit(*commit_args)
+        else:
+            s3 = L.orthrus_consensus(*cons_args)
         if ev is not None:
             ev[3].record(stream)
-        s4 = L.orthrus_kv_append(*app_args)
+        s4 = 0 if write else L.orthrus_kv_append(*app_args)
         if ev is not None:
             ev[4].record(stream)
         if s1 or s2 or s3 or s4:
@@ -425,7 +434,11 @@ def run_ours(args):
             "block_attn_gbs": attn_gbs, "block_attn_us": {"diffusion": t_diff * 1e3,
                                                           "verify": t_ver * 1e3},
             "consensus_rows_per_s": world * m.R / (t_cons * 1e-3),
-            "consensus_us": t_cons * 1e3, "kv_append_us": t_app * 1e3,
+            "consensus_us": t_cons * 1e3,
+            "kv_append_us": None if write else t_app * 1e3,
+            "commit": ("write-then-truncate (VERIFY attention stores the block K/V; "
+                       "consensus advances the lengths)") if write else
+                      "separate kv_append of the accepted rows",
             "blocks_per_s": world * m.B / (ms_step * 1e-3),
             "tokens_verified_per_s": world * m.R / (t_ver * 1e-3),
             "mean_accept_len": mean_accept,
@@ -455,6 +468,9 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--commit", choices=["write", "append"], default="write",
+                    help="write: VERIFY attention stores the block K/V and consensus advances "
+                         "the lengths (write-then-truncate); append: separate kv_append launch")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -16,7 +16,7 @@
 // the prefix lengths; a unit cut by a range boundary is finished by the combine
 // kernel from per-CTA partials (max, sum, normalised accumulator).
 //
-// Roles (352 threads):
+// Roles (384 threads):
 //   warp 0      TMA producer, two lanes: lane 0 issues the Q tile per unit
 //               and the K tiles into a K ring, lane 1 the V tiles into a
 //               separate, deeper V ring (K is released by its QK three tiles
@@ -33,6 +33,9 @@
 //               its S row for the PV MMA (A operand from TMEM) and, at the
 //               end of a unit, merges the two groups'
 //               accumulators and stores the output (or a partial).
+//   warp 11     block writer (write-then-truncate VERIFY only): copies the
+//               block's K/V rows into the cache slots after the prefix while
+//               the pipeline streams that prefix; otherwise idle.
 // The two softmax groups keep separate O accumulators (TMEM columns), so they
 // never wait on each other inside a unit.
 #pragma once
@@ -48,10 +51,11 @@ namespace orthrus {
 
 constexpr int kTileN = 64;          // keys per tile
 constexpr int kTileM = 128;         // query rows per MMA tile
-constexpr int kAttnThreads = 352;   // 11 warps
+constexpr int kAttnThreads = 384;   // 12 warps
 constexpr int kProducerWarp = 0;
 constexpr int kMmaWarp0 = 1;        // warps 1 and 2 issue the MMAs of softmax groups 0 and 1
 constexpr int kSoftmaxWarp0 = 3;    // warps 3-6: softmax group 0, warps 7-10: group 1
+constexpr int kWriterWarp = 11;     // block K/V -> cache (write-then-truncate VERIFY)
 constexpr uint32_t kTmemCols = 512;
 constexpr int kSPerGroup = 2;       // S buffers per group: QK runs one own tile ahead
 constexpr uint32_t kTmemS = 0;      // S buffer k of group w at column 64*(2w + k)
@@ -77,6 +81,13 @@ struct AttnArgs {
   unsigned long long timeout_ns;
   int fault_inject;  // test hook: 1 drops each CTA's first V copy (a wait must time out)
   int out_v8;        // out is 32-byte aligned: rows are written with 256-bit stores
+  // Write-then-truncate VERIFY: also store block rows [0, K_b) of k/v_block
+  // into the cache slots L_b .. L_b + K_b - 1 (the caller commits L_b += n_b).
+  int write_block;
+  const uint4* kb_rows;  // k_block / v_block as 16-byte chunks
+  const uint4* vb_rows;
+  uint4* kc_rows;        // k_cache / v_cache as 16-byte chunks
+  uint4* vc_rows;
 };
 
 // ---------------------------------------------------------------------------
@@ -948,6 +959,68 @@ __device__ __forceinline__ void softmax_role(const AttnArgs& a, uint8_t* smem, u
   }
 }
 
+// Block writer (write-then-truncate VERIFY: the AR view writes every block
+// row's K/V into the cache as it verifies the block, and the commit only moves
+// the prefix length; technical summary §2.3 item 3). For each unit of this
+// CTA's range whose block tile the CTA owns, block row i of head h goes to the
+// cache slot of position L_b + i. These slots lie past every key the call
+// reads from the cache (the prefix ends at L_b; a partial last prefix tile
+// masks keys at or past L_b and zeroes their V rows), so the copy runs next to
+// the pipeline with no ordering against it. A row whose page index or page id
+// is out of range is skipped and flagged. No waits.
+template <int D>
+__device__ __forceinline__ void block_writer_role(const AttnArgs& a, const SeqTable& tab,
+                                                  SegCursor c) {
+  constexpr int kChunks = D / 8;  // 16-byte chunks per head row
+  constexpr int U = 8;            // chunk pairs in flight per lane
+  const int lane = threadIdx.x & 31;
+  Segment sg;
+  while (cursor_next(a, tab, c, sg)) {
+    if (sg.t1 != sg.nt) continue;  // another CTA owns this unit's block tile
+    const SeqInfo si = tab.get(a, sg.b);
+    const int items = si.Kb * kChunks;
+    const int* table = a.page_table + (long long)sg.b * a.max_pages;
+    for (int base = lane; base < items; base += 32 * U) {
+      uint4 kv[U], vv[U];
+      long long dst[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int e = base + 32 * u;
+        dst[u] = -1;
+        if (e < items) {
+          const int i = e / kChunks, ch = e % kChunks;
+          const long long pos = (long long)si.L + i;
+          const long long pidx = pos / a.page_size;
+          int page = -1;
+          if (pidx >= a.max_pages) {
+            raise_flag(a, ORTHRUS_FLAG_BAD_LENGTH);
+          } else {
+            page = table[pidx];
+            if (page < 0 || page >= a.num_pages) {
+              raise_flag(a, ORTHRUS_FLAG_BAD_PAGE);
+              page = -1;
+            }
+          }
+          if (page >= 0) {
+            const long long src = ((long long)(si.row0 + i) * a.Hkv + sg.h) * kChunks + ch;
+            dst[u] = (((long long)page * a.Hkv + sg.h) * a.page_size + pos % a.page_size) *
+                         kChunks + ch;
+            kv[u] = a.kb_rows[src];
+            vv[u] = a.vb_rows[src];
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        if (dst[u] >= 0) {
+          a.kc_rows[dst[u]] = kv[u];
+          a.vc_rows[dst[u]] = vv[u];
+        }
+      }
+    }
+  }
+}
+
 template <int D>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     block_attn_kernel(const __grid_constant__ CUtensorMap tm_q,
@@ -1018,6 +1091,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       producer_role<D>(a, smem, &tm_q, &tm_kc, &tm_vc, &tm_kb, &tm_vb, abort_flag, tab, start);
   } else if (warp < kSoftmaxWarp0) {
     mma_role<D>(a, smem, tmem, abort_flag, warp - kMmaWarp0, tab, start);
+  } else if (warp == kWriterWarp) {
+    if (a.write_block) block_writer_role<D>(a, tab, start);
   } else {
     softmax_role<D>(a, smem, tmem, abort_flag, tab, start);
   }

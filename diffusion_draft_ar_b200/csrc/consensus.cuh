@@ -137,7 +137,8 @@ __global__ void consensus_finalize_kernel(const unsigned long long* __restrict__
                                           const int* __restrict__ cu_block, int B, int max_block,
                                           int* __restrict__ accept_len,
                                           int* __restrict__ next_token,
-                                          int* __restrict__ row_argmax) {
+                                          int* __restrict__ row_argmax,
+                                          int* __restrict__ prefix_lens) {
   const int warps = blockDim.x >> 5;
   const int b = blockIdx.x * warps + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
@@ -178,6 +179,9 @@ __global__ void consensus_finalize_kernel(const unsigned long long* __restrict__
     const int n = (m + 1 < Kb) ? (m + 1) : Kb;
     accept_len[b] = n;
     next_token[b] = next;
+    // Commit of write-then-truncate VERIFY: the cache already holds all K_b
+    // rows past L_b, so accepting n of them is advancing the length.
+    if (prefix_lens) prefix_lens[b] += n;
   }
 }
 

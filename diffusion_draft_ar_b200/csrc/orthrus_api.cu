@@ -190,7 +190,7 @@ orthrus_status_t plan_attn(const orthrus_attn_params* p, int sms, AttnPlan* pl) 
 
 template <int D>
 orthrus_status_t launch_attn(const orthrus_attn_params* p, const AttnPlan& pl, int dev,
-                             cudaStream_t stream) {
+                             cudaStream_t stream, bool write_block) {
   using Lay = AttnLayout<D>;
   static std::atomic<int> smem_set[kMaxDevices];
   if (!smem_set[dev].load()) {
@@ -262,6 +262,12 @@ orthrus_status_t launch_attn(const orthrus_attn_params* p, const AttnPlan& pl, i
     a.fault_inject = fi ? std::atoi(fi) : 0;
   }
   a.out_v8 = aligned(p->out, 32) ? 1 : 0;
+  a.write_block = write_block ? 1 : 0;
+  a.kb_rows = static_cast<const uint4*>(p->k_block);
+  a.vb_rows = static_cast<const uint4*>(p->v_block);
+  // The write-then-truncate entry point documents that the cache is written.
+  a.kc_rows = static_cast<uint4*>(const_cast<void*>(p->k_cache));
+  a.vc_rows = static_cast<uint4*>(const_cast<void*>(p->v_cache));
 
   block_attn_kernel<D><<<pl.grid, kAttnThreads, Lay::kAlloc, stream>>>(tq, tkc, tvc, tkb, tvb, a);
   cudaError_t e = cudaGetLastError();
@@ -311,7 +317,7 @@ int32_t orthrus_block_attn_kernel_count(const orthrus_attn_params* p) {
   return pl.combine ? 2 : 1;
 }
 
-orthrus_status_t orthrus_block_attn(const orthrus_attn_params* p, void* stream) {
+static orthrus_status_t block_attn_entry(const orthrus_attn_params* p, void* stream, bool write_block) {
   AttnPlan pl;
   orthrus_status_t s = plan_attn(p, 1, &pl);  // geometry checks first, no CUDA call
   if (s != ORTHRUS_OK) return s;
@@ -343,7 +349,18 @@ orthrus_status_t orthrus_block_attn(const orthrus_attn_params* p, void* stream) 
     return fail(ORTHRUS_ERR_INVALID_ARG, "workspace %zu bytes < %zu needed", p->workspace_bytes,
                 pl.ws_bytes);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  return p->D == 128 ? launch_attn<128>(p, pl, dev, st) : launch_attn<64>(p, pl, dev, st);
+  return p->D == 128 ? launch_attn<128>(p, pl, dev, st, write_block)
+                     : launch_attn<64>(p, pl, dev, st, write_block);
+}
+
+orthrus_status_t orthrus_block_attn(const orthrus_attn_params* p, void* stream) {
+  return block_attn_entry(p, stream, false);
+}
+
+orthrus_status_t orthrus_block_attn_verify_write(const orthrus_attn_params* p, void* stream) {
+  if (p && p->view != ORTHRUS_VIEW_VERIFY)
+    return fail(ORTHRUS_ERR_INVALID_ARG, "write-then-truncate needs the VERIFY view");
+  return block_attn_entry(p, stream, true);
 }
 
 size_t orthrus_consensus_workspace_size(int32_t B, int32_t max_block, int32_t V) {
@@ -352,11 +369,12 @@ size_t orthrus_consensus_workspace_size(int32_t B, int32_t max_block, int32_t V)
   return static_cast<size_t>(B) * max_block * chunks * sizeof(unsigned long long);
 }
 
-orthrus_status_t orthrus_consensus(const float* verify_logits, int64_t ld, int32_t V,
-                                   const int32_t* draft_tokens, const int32_t* cu_block,
-                                   int32_t B, int32_t max_block, int32_t* accept_len,
-                                   int32_t* next_token, int32_t* row_argmax, void* workspace,
-                                   size_t workspace_bytes, void* stream) {
+static orthrus_status_t consensus_entry(const float* verify_logits, int64_t ld, int32_t V,
+                                        const int32_t* draft_tokens, const int32_t* cu_block,
+                                        int32_t B, int32_t max_block, int32_t* accept_len,
+                                        int32_t* next_token, int32_t* row_argmax,
+                                        int32_t* prefix_lens, void* workspace,
+                                        size_t workspace_bytes, void* stream) {
   if (B < 0) return fail(ORTHRUS_ERR_INVALID_ARG, "B = %d < 0", B);
   if (V < 1 || ld < V) return fail(ORTHRUS_ERR_INVALID_ARG, "V = %d, ld = %lld", V, (long long)ld);
   if (max_block < 1) return fail(ORTHRUS_ERR_INVALID_ARG, "max_block = %d", max_block);
@@ -393,9 +411,30 @@ orthrus_status_t orthrus_consensus(const float* verify_logits, int64_t ld, int32
   cfg.numAttrs = 1;
   e = cudaLaunchKernelEx(&cfg, consensus_finalize_kernel, static_cast<const unsigned long long*>(part),
                          n_chunks, draft_tokens, cu_block, static_cast<int>(B),
-                         static_cast<int>(max_block), accept_len, next_token, row_argmax);
+                         static_cast<int>(max_block), accept_len, next_token, row_argmax,
+                         prefix_lens);
   if (e != cudaSuccess) return fail(ORTHRUS_ERR_CUDA, "consensus launch: %s", cudaGetErrorString(e));
   return ok();
+}
+
+orthrus_status_t orthrus_consensus(const float* verify_logits, int64_t ld, int32_t V,
+                                   const int32_t* draft_tokens, const int32_t* cu_block,
+                                   int32_t B, int32_t max_block, int32_t* accept_len,
+                                   int32_t* next_token, int32_t* row_argmax, void* workspace,
+                                   size_t workspace_bytes, void* stream) {
+  return consensus_entry(verify_logits, ld, V, draft_tokens, cu_block, B, max_block, accept_len,
+                         next_token, row_argmax, nullptr, workspace, workspace_bytes, stream);
+}
+
+orthrus_status_t orthrus_consensus_commit(const float* verify_logits, int64_t ld, int32_t V,
+                                          const int32_t* draft_tokens, const int32_t* cu_block,
+                                          int32_t B, int32_t max_block, int32_t* accept_len,
+                                          int32_t* next_token, int32_t* row_argmax,
+                                          int32_t* prefix_lens, void* workspace,
+                                          size_t workspace_bytes, void* stream) {
+  if (B > 0 && !prefix_lens) return fail(ORTHRUS_ERR_INVALID_ARG, "prefix_lens is NULL");
+  return consensus_entry(verify_logits, ld, V, draft_tokens, cu_block, B, max_block, accept_len,
+                         next_token, row_argmax, prefix_lens, workspace, workspace_bytes, stream);
 }
 
 orthrus_status_t orthrus_kv_append(const void* k_block, const void* v_block,
@@ -495,7 +534,7 @@ orthrus_status_t orthrus_consensus_noalloc(const float* verify_logits, int64_t l
   const int warps = 8;
   consensus_finalize_kernel<<<(B + warps - 1) / warps, warps * 32, 0, st>>>(
       part, static_cast<int>(n_chunks), draft_tokens, cu_block, B, max_block, accept_len,
-      next_token, row_argmax);
+      next_token, row_argmax, nullptr);
   e = cudaGetLastError();
   if (e != cudaSuccess) return fail(ORTHRUS_ERR_CUDA, "consensus launch: %s", cudaGetErrorString(e));
   return ok();

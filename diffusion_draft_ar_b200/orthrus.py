@@ -52,10 +52,15 @@ lib.orthrus_block_attn_kernel_count.restype = _i32
 lib.orthrus_block_attn_kernel_count.argtypes = [ctypes.POINTER(AttnParams)]
 lib.orthrus_block_attn.restype = _i32
 lib.orthrus_block_attn.argtypes = [ctypes.POINTER(AttnParams), _vp]
+lib.orthrus_block_attn_verify_write.restype = _i32
+lib.orthrus_block_attn_verify_write.argtypes = [ctypes.POINTER(AttnParams), _vp]
 lib.orthrus_consensus_workspace_size.restype = _sz
 lib.orthrus_consensus_workspace_size.argtypes = [_i32, _i32, _i32]
 lib.orthrus_consensus.restype = _i32
 lib.orthrus_consensus.argtypes = [_vp, _i64, _i32, _vp, _vp, _i32, _i32, _vp, _vp, _vp, _vp, _sz, _vp]
+lib.orthrus_consensus_commit.restype = _i32
+lib.orthrus_consensus_commit.argtypes = [_vp, _i64, _i32, _vp, _vp, _i32, _i32, _vp, _vp, _vp, _vp,
+                                         _vp, _sz, _vp]
 lib.orthrus_kv_append.restype = _i32
 lib.orthrus_kv_append.argtypes = [_vp, _vp, _vp, _i32, _vp, _vp, _i32, _vp, _i32, _i32, _vp, _vp,
                                   _i32, _i32, _i32, _i32, _vp, _vp]
@@ -158,13 +163,30 @@ def block_attn(view, q_block, k_cache, v_cache, k_block, v_block, prefix_lens, c
     return out
 
 
+def block_attn_verify_write(q_block, k_cache, v_cache, k_block, v_block, prefix_lens, cu_block,
+                            page_table, out, workspace, max_block: int, softmax_scale: float = 0.0,
+                            kv_split_tokens: int = 0, max_ctas: int = 0, error_flag=None,
+                            stream=None):
+    """``orthrus_block_attn_verify_write``: VERIFY attention that also stores every
+    block row's K/V past each prefix (k_cache / v_cache written in place; the
+    lengths are left for ``consensus_commit``)."""
+    p = attn_params("verify", q_block, k_cache, v_cache, k_block, v_block, prefix_lens,
+                    cu_block, page_table, out, max_block, workspace, softmax_scale,
+                    kv_split_tokens, max_ctas, error_flag)
+    _check(lib.orthrus_block_attn_verify_write(ctypes.byref(p), _stream(stream)),
+           "orthrus_block_attn_verify_write")
+    return out
+
+
 def consensus_workspace_size(B: int, max_block: int, V: int) -> int:
     return int(lib.orthrus_consensus_workspace_size(B, max_block, V))
 
 
 def consensus(verify_logits, draft_tokens, cu_block, B: int, max_block: int, accept_len,
-              next_token, workspace, row_argmax=None, stream=None):
-    """``orthrus_consensus``: writes accept_len, next_token (and row_argmax) in place."""
+              next_token, workspace, row_argmax=None, stream=None, prefix_lens=None):
+    """``orthrus_consensus``: writes accept_len, next_token (and row_argmax) in place.
+    With ``prefix_lens`` it is ``orthrus_consensus_commit``: the lengths also
+    advance by the accepted counts (after ``block_attn_verify_write``)."""
     if not verify_logits.is_cuda or verify_logits.dtype != torch.float32 or verify_logits.dim() != 2:
         raise ValueError("verify_logits must be a 2-D CUDA float32 tensor")
     if verify_logits.stride(1) != 1:
@@ -178,6 +200,15 @@ def consensus(verify_logits, draft_tokens, cu_block, B: int, max_block: int, acc
     if row_argmax is not None:
         _need(row_argmax, "row_argmax", torch.int32, 1)
     V = verify_logits.shape[1]
+    if prefix_lens is not None:
+        _need(prefix_lens, "prefix_lens", torch.int32, 1)
+        st = lib.orthrus_consensus_commit(_ptr(verify_logits), verify_logits.stride(0), V,
+                                          _ptr(draft_tokens), _ptr(cu_block), int(B),
+                                          int(max_block), _ptr(accept_len), _ptr(next_token),
+                                          _ptr(row_argmax), _ptr(prefix_lens), _ptr(workspace),
+                                          workspace.numel(), _stream(stream))
+        _check(st, "orthrus_consensus_commit")
+        return
     st = lib.orthrus_consensus(_ptr(verify_logits), verify_logits.stride(0), V, _ptr(draft_tokens),
                                _ptr(cu_block), int(B), int(max_block), _ptr(accept_len),
                                _ptr(next_token), _ptr(row_argmax), _ptr(workspace),

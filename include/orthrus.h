@@ -147,6 +147,34 @@ ORTHRUS_API int32_t orthrus_block_attn_kernel_count(const orthrus_attn_params* p
 ORTHRUS_API orthrus_status_t orthrus_block_attn(const orthrus_attn_params* p, void* stream);
 
 /*
+ * Write-then-truncate VERIFY (technical summary §2.3 item 3: the AR view
+ * writes the whole block's KV while it verifies it, and the commit truncates
+ * the cache to the accepted prefix). Same attention as orthrus_block_attn with
+ * p->view == ORTHRUS_VIEW_VERIFY and, in the same launch, for every sequence
+ * b, block row i in [0, K_b) and KV head h, with L_b = prefix_lens[b]:
+ *
+ *   k_cache[page_table[b][(L_b+i)/P], h, (L_b+i) % P, :] = k_block[row0_b + i, h, :]
+ *
+ * and the same for V. prefix_lens is not changed: orthrus_consensus_commit
+ * then advances it by the accepted count, which leaves the cache bytes of
+ * every position below the new length identical to orthrus_block_attn
+ * followed by orthrus_kv_append, and removes the append launch. Slots
+ * L_b + n_b .. L_b + K_b - 1 keep the rejected rows until the next round
+ * overwrites them (they lie past the committed length).
+ *   - k_cache and v_cache are WRITTEN through the params' const pointers.
+ *   - The page table must reach position L_b + K_b - 1; a row past it is
+ *     skipped and flags ORTHRUS_FLAG_BAD_LENGTH, a row whose page id is out of
+ *     range is skipped and flags ORTHRUS_FLAG_BAD_PAGE. A raised flag means
+ *     the round's cache is incomplete: do not commit it.
+ *   - The slots written must not be read by any sequence of the same call
+ *     (pages holding positions >= L_b are not shared with another sequence's
+ *     prefix).
+ * Errors: as orthrus_block_attn; INVALID_ARG when p->view is not VERIFY.
+ */
+ORTHRUS_API orthrus_status_t orthrus_block_attn_verify_write(const orthrus_attn_params* p,
+                                                             void* stream);
+
+/*
  * Greedy consensus (technical summary §2.3 item 3: a drafted token is accepted
  * iff it equals the frozen AR view's greedy token, checked left to right; at the
  * first divergence j the prefix up to j-1 is committed and the exact AR
@@ -173,6 +201,24 @@ ORTHRUS_API orthrus_status_t orthrus_consensus(const float* verify_logits, int64
                                    int32_t B, int32_t max_block, int32_t* accept_len,
                                    int32_t* next_token, int32_t* row_argmax, void* workspace,
                                    size_t workspace_bytes, void* stream);
+
+/*
+ * Consensus plus the commit of write-then-truncate VERIFY (technical summary
+ * §2.3 item 3). Same operation, arguments and results as orthrus_consensus,
+ * and in the same launches prefix_lens[b] += accept_len[b] for every sequence
+ * (a sequence with K_b = 0 is left unchanged). Meant to follow
+ * orthrus_block_attn_verify_write, which already stored all K_b block rows
+ * past L_b: advancing the length is then the whole commit.
+ *   prefix_lens  device int32 [B], updated in place (required)
+ * Errors: as orthrus_consensus; INVALID_ARG when prefix_lens is NULL.
+ */
+ORTHRUS_API orthrus_status_t orthrus_consensus_commit(const float* verify_logits, int64_t ld,
+                                                      int32_t V, const int32_t* draft_tokens,
+                                                      const int32_t* cu_block, int32_t B,
+                                                      int32_t max_block, int32_t* accept_len,
+                                                      int32_t* next_token, int32_t* row_argmax,
+                                                      int32_t* prefix_lens, void* workspace,
+                                                      size_t workspace_bytes, void* stream);
 
 /*
  * Commit (technical summary §2.3 item 3, commit the synchronised prefix and

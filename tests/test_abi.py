@@ -158,3 +158,33 @@ def test_kv_append_rejects_bad_arguments(O, args):
                                  a["lens"], 1, a["table"], 4, 8, a["k_cache"], a["v_cache"],
                                  a["B"], a["Hkv"], a["D"], a["page_size"], None, None)
     assert st == 1
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(view=0), 1), (dict(view=2), 1), (dict(D=96), 2), (dict(q_block=None), 1),
+    (dict(k_cache=0x20008), 1), (dict(workspace=None), 1),
+])
+def test_block_attn_verify_write_rejects_bad_arguments(O, kw, status):
+    # write-then-truncate runs the VERIFY view only; the rest as orthrus_block_attn
+    p = _params(O, **kw)
+    assert O.lib.orthrus_block_attn_verify_write(ctypes.byref(p), None) == status
+    assert O.lib.orthrus_last_error() != b""
+
+
+def test_block_attn_verify_write_empty_batch_is_a_no_op(O):
+    p = _params(O, B=0, q_block=None, out=None)
+    assert O.lib.orthrus_block_attn_verify_write(ctypes.byref(p), None) == 0
+
+
+@pytest.mark.parametrize("args,status", [
+    (dict(lens=None), 1), (dict(V=0), 1), (dict(workspace=None), 1), (dict(logits=0x10002), 1),
+])
+def test_consensus_commit_rejects_bad_arguments(O, args, status):
+    a = dict(logits=0x10000, ld=512, V=512, draft=0x20000, cu=None, B=2, max_block=8,
+             acc=0x30000, nxt=0x40000, am=None, lens=0x60000, workspace=0x50000,
+             workspace_bytes=1 << 20)
+    a.update(args)
+    st = O.lib.orthrus_consensus_commit(a["logits"], a["ld"], a["V"], a["draft"], a["cu"], a["B"],
+                                        a["max_block"], a["acc"], a["nxt"], a["am"], a["lens"],
+                                        a["workspace"], a["workspace_bytes"], None)
+    assert st == status
