@@ -23,6 +23,11 @@ Dual-View Diffusion, technical summary):
 * ``kv_append`` -- §2.3 item 3 (commit and truncate the cache) and the
   agents-report.net commentary, "core design" (accepted tokens' KV appended to
   the shared cache).
+* ``lm_head_logits`` / ``greedy_tokens`` -- §2.3 items 2-3 with §2.1: the
+  frozen AR model's output projection scores each block row over the
+  vocabulary, and its greedy token is the first index of the largest score.
+* ``accept_from_tokens`` -- the §2.3 item 3 rule of ``consensus`` applied to
+  given greedy tokens.
 """
 from __future__ import annotations
 
@@ -78,6 +83,12 @@ def _load():
         lib.oracle_consensus.argtypes = [p, i64, i32, p, p, i32, p, p, p, i32]
         lib.oracle_kv_append.restype = i32
         lib.oracle_kv_append.argtypes = [p, p, p, p, p, i32, p, i32, i32, p, p, i32, i32, i32, i32]
+        lib.oracle_accept.restype = None
+        lib.oracle_accept.argtypes = [p, p, p, i32, p, p]
+        lib.oracle_lm_head.restype = i32
+        lib.oracle_lm_head.argtypes = [p, p, i32, i32, p, i64, p, p, i32]
+        lib.oracle_greedy_tokens.restype = None
+        lib.oracle_greedy_tokens.argtypes = [p, i64, i32, p]
         _lib = lib
         return lib
 
@@ -211,3 +222,54 @@ def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
     """Exact widening of bf16 bit patterns (uint16) to float64."""
     u = np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16
     return u.view(np.float32).astype(np.float64)
+
+
+def accept_from_tokens(tokens, draft_tokens, cu_block):
+    """The consensus rule on given greedy tokens: (accept_len[B], next_token[B])."""
+    lib = _load()
+    t = _c(tokens, np.int32)
+    dr = _c(draft_tokens, np.int32)
+    cu = _c(cu_block, np.int32)
+    B = cu.shape[0] - 1
+    if t.shape[0] < int(cu[-1]) or dr.shape[0] < int(cu[-1]):
+        raise ValueError("inconsistent accept shapes")
+    acc = np.zeros(B, np.int32)
+    nxt = np.zeros(B, np.int32)
+    lib.oracle_accept(_ptr(t), _ptr(dr), _ptr(cu), B, _ptr(acc), _ptr(nxt))
+    return acc, nxt
+
+
+def lm_head_logits(hidden, w_head, rows=None, with_absdot: bool = False,
+                   threads: int | None = None):
+    """fp64 scores of the AR view's LM head: logits[i, v] = <hidden[rows[i]], w_head[v]>.
+
+    ``hidden`` [R, d] and ``w_head`` [V, d] are bf16 bit patterns (uint16).
+    Returns logits [n, V] (and, with ``with_absdot``, the sums of |products|).
+    """
+    lib = _load()
+    h = _c(hidden, np.uint16)
+    w = _c(w_head, np.uint16)
+    if h.ndim != 2 or w.ndim != 2 or h.shape[1] != w.shape[1]:
+        raise ValueError("hidden [R, d] and w_head [V, d] expected")
+    R, d = h.shape
+    V = w.shape[0]
+    r = np.arange(R, dtype=np.int64) if rows is None else _c(rows, np.int64)
+    if r.size and (r.min() < 0 or r.max() >= R):
+        raise ValueError("row index out of range")
+    out = np.empty((r.shape[0], V), np.float64)
+    ab = np.empty((r.shape[0], V), np.float64) if with_absdot else None
+    rc = lib.oracle_lm_head(_ptr(h), _ptr(w), d, V, _ptr(r), r.shape[0], _ptr(out), _ptr(ab),
+                            threads or default_threads())
+    if rc != 0:
+        raise ValueError(f"oracle_lm_head: bad input (code {rc})")
+    return (out, ab) if with_absdot else out
+
+
+def greedy_tokens(logits64):
+    """First index of the largest fp64 score per row (NaN as -inf)."""
+    lib = _load()
+    x = _c(logits64, np.float64)
+    n, V = x.shape
+    t = np.zeros(n, np.int32)
+    lib.oracle_greedy_tokens(_ptr(x), n, V, _ptr(t))
+    return t

@@ -24,6 +24,13 @@
  *     commit up to j-1 and append the AR correction token).
  *   - oracle_kv_append: technical summary §2.3 item 3 ("truncates the cache")
  *     and the commentary's "appends their KV state to the shared cache".
+ *   - oracle_lm_head, oracle_greedy_tokens: technical summary §2.3 items 2-3
+ *     (the frozen AR view scores the populated block; its greedy token per row
+ *     is the largest of those scores). The scores are the AR model's output
+ *     projection of each row's final hidden state (technical summary §2.1: the
+ *     AR view is the unchanged base model).
+ *   - oracle_accept: the left-to-right rule of oracle_consensus on given
+ *     greedy tokens (technical summary §2.3 item 3).
  *
  * Layouts (all row-major, caller-owned host memory):
  *   q_block  [R, Hq, D]                   bf16 bits (uint16)
@@ -334,20 +341,13 @@ static void argmax_row(void* ctx, int64_t r) {
  *   n_b  = min(m_b + 1, K_b)     (accepted drafts plus the AR correction)
  *   next = t_{row0 + n_b - 1}    (the token that becomes the next anchor)
  * A sequence with K_b = 0 gets n_b = 0 and next = -1. row_argmax may be NULL. */
-int oracle_consensus(const float* logits, int64_t ld, int V, const int32_t* draft,
-                     const int32_t* cu_block, int B, int32_t* accept_len, int32_t* next_token,
-                     int32_t* row_argmax, int threads) {
-  if (V < 1 || ld < V || B < 0) return -1;
-  int64_t R = (B > 0) ? cu_block[B] : 0;
-  int32_t* t = row_argmax;
-  int32_t* own = NULL;
-  if (!t) {
-    own = (int32_t*)malloc(sizeof(int32_t) * (size_t)(R > 0 ? R : 1));
-    if (!own) return -2;
-    t = own;
-  }
-  argmax_job a = {logits, ld, V, t};
-  parallel_for(R, argmax_row, &a, threads);
+/* For each sequence b with block rows row0 .. row0+K_b-1 and greedy tokens t:
+ *   m_b  = number of leading rows whose draft equals t_r
+ *   n_b  = min(m_b + 1, K_b)     (accepted drafts plus the AR correction)
+ *   next = t_{row0 + n_b - 1}    (the token that becomes the next anchor)
+ * A sequence with K_b = 0 gets n_b = 0 and next = -1. */
+void oracle_accept(const int32_t* t, const int32_t* draft, const int32_t* cu_block, int B,
+                   int32_t* accept_len, int32_t* next_token) {
   for (int b = 0; b < B; ++b) {
     int64_t row0 = cu_block[b];
     int64_t Kb = (int64_t)cu_block[b + 1] - row0;
@@ -362,6 +362,23 @@ int oracle_consensus(const float* logits, int64_t ld, int V, const int32_t* draf
     accept_len[b] = (int32_t)n;
     next_token[b] = t[row0 + n - 1];
   }
+}
+
+int oracle_consensus(const float* logits, int64_t ld, int V, const int32_t* draft,
+                     const int32_t* cu_block, int B, int32_t* accept_len, int32_t* next_token,
+                     int32_t* row_argmax, int threads) {
+  if (V < 1 || ld < V || B < 0) return -1;
+  int64_t R = (B > 0) ? cu_block[B] : 0;
+  int32_t* t = row_argmax;
+  int32_t* own = NULL;
+  if (!t) {
+    own = (int32_t*)malloc(sizeof(int32_t) * (size_t)(R > 0 ? R : 1));
+    if (!own) return -2;
+    t = own;
+  }
+  argmax_job a = {logits, ld, V, t};
+  parallel_for(R, argmax_row, &a, threads);
+  oracle_accept(t, draft, cu_block, B, accept_len, next_token);
   free(own);
   return 0;
 }
@@ -418,4 +435,73 @@ int oracle_kv_append(const uint16_t* k_block, const uint16_t* v_block, const int
     bad |= seq_bad;
   }
   return bad;
+}
+
+/* ------------------------------------------------------------------------- */
+/* LM head: the AR view's scores of the block rows                            */
+
+typedef struct {
+  const uint16_t* hidden;  /* [R, d] bf16 bits */
+  const uint16_t* w;       /* [V, d] bf16 bits, one row per vocabulary entry */
+  int d, V;
+  const int64_t* rows;     /* the rows of hidden to score */
+  double* logits;          /* [nrows, V] */
+  double* absdot;          /* [nrows, V] or NULL */
+  int64_t vchunk, n_vchunks;
+} lmhead_job;
+
+/* logits[i, v] = sum_k hidden[rows[i], k] * w[v, k], and absdot[i, v] =
+ * sum_k |hidden[rows[i], k] * w[v, k]| (the scale of the rounding error of any
+ * shorter-precision evaluation of the same sum). Every bf16 product is exact
+ * in double; the sum runs over k in increasing order. */
+static void lmhead_task(void* ctx, int64_t task) {
+  lmhead_job* a = (lmhead_job*)ctx;
+  int64_t i = task / a->n_vchunks;
+  int64_t c = task % a->n_vchunks;
+  const uint16_t* h = a->hidden + a->rows[i] * (int64_t)a->d;
+  int64_t v0 = c * a->vchunk;
+  int64_t v1 = v0 + a->vchunk < a->V ? v0 + a->vchunk : a->V;
+  double* hv = (double*)malloc(sizeof(double) * (size_t)a->d);
+  if (!hv) return;
+  for (int k = 0; k < a->d; ++k) hv[k] = bf16_to_double(h[k]);
+  for (int64_t v = v0; v < v1; ++v) {
+    const uint16_t* wr = a->w + v * (int64_t)a->d;
+    double s = 0.0, sa = 0.0;
+    for (int k = 0; k < a->d; ++k) {
+      double x = hv[k] * bf16_to_double(wr[k]);
+      s += x;
+      sa += fabs(x);
+    }
+    a->logits[i * (int64_t)a->V + v] = s;
+    if (a->absdot) a->absdot[i * (int64_t)a->V + v] = sa;
+  }
+  free(hv);
+}
+
+int oracle_lm_head(const uint16_t* hidden, const uint16_t* w_head, int d_model, int V,
+                   const int64_t* rows, int64_t nrows, double* logits, double* absdot,
+                   int threads) {
+  if (d_model < 1 || V < 1 || nrows < 0) return -1;
+  lmhead_job a = {hidden, w_head, d_model, V, rows, logits, absdot, 4096, 0};
+  a.n_vchunks = (V + a.vchunk - 1) / a.vchunk;
+  parallel_for(nrows * a.n_vchunks, lmhead_task, &a, threads);
+  return 0;
+}
+
+/* Greedy token of each row of fp64 scores [nrows, V]: the first index holding
+ * the largest value (NaN counts as -inf, -0 == +0). */
+void oracle_greedy_tokens(const double* logits, int64_t nrows, int V, int32_t* t) {
+  for (int64_t i = 0; i < nrows; ++i) {
+    const double* x = logits + i * (int64_t)V;
+    double best = -INFINITY;
+    int32_t idx = 0;
+    for (int v = 0; v < V; ++v) {
+      double xv = isnan(x[v]) ? -INFINITY : x[v];
+      if (xv > best) {
+        best = xv;
+        idx = v;
+      }
+    }
+    t[i] = idx;
+  }
 }
