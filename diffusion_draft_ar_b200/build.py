@@ -19,7 +19,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "liborthrus.so")
 SOURCES = ["orthrus_api.cu"]
-HEADERS = ["block_attn.cuh", "consensus.cuh", "kv_append.cuh", "ptx.cuh"]
+HEADERS = ["block_attn.cuh", "consensus.cuh", "kv_append.cuh", "lm_head.cuh", "ptx.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -138,14 +138,15 @@ __global__ void consensus_finalize_kernel(const unsigned long long* __restrict__
                                           int* __restrict__ accept_len,
                                           int* __restrict__ next_token,
                                           int* __restrict__ row_argmax,
-                                          int* __restrict__ prefix_lens) {
+                                          int* __restrict__ prefix_lens, int row_limit) {
   const int warps = blockDim.x >> 5;
   const int b = blockIdx.x * warps + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (b >= B) return;
   const int row0 = cu_block ? cu_block[b] : b * max_block;
   const int Kb = cu_block ? cu_block[b + 1] - row0 : max_block;
-  if (Kb <= 0) {
+  // rows outside the keys the caller's workspace holds: treated as an empty block
+  if (Kb <= 0 || row0 < 0 || row0 + Kb > row_limit) {
     if (lane == 0) {
       accept_len[b] = 0;
       next_token[b] = -1;

@@ -16,6 +16,7 @@
 #include "block_attn.cuh"
 #include "consensus.cuh"
 #include "kv_append.cuh"
+#include "lm_head.cuh"
 #include "orthrus.h"
 
 namespace {
@@ -412,7 +413,7 @@ static orthrus_status_t consensus_entry(const float* verify_logits, int64_t ld, 
   e = cudaLaunchKernelEx(&cfg, consensus_finalize_kernel, static_cast<const unsigned long long*>(part),
                          n_chunks, draft_tokens, cu_block, static_cast<int>(B),
                          static_cast<int>(max_block), accept_len, next_token, row_argmax,
-                         prefix_lens);
+                         prefix_lens, static_cast<int>(R_max));
   if (e != cudaSuccess) return fail(ORTHRUS_ERR_CUDA, "consensus launch: %s", cudaGetErrorString(e));
   return ok();
 }
@@ -534,7 +535,7 @@ orthrus_status_t orthrus_consensus_noalloc(const float* verify_logits, int64_t l
   const int warps = 8;
   consensus_finalize_kernel<<<(B + warps - 1) / warps, warps * 32, 0, st>>>(
       part, static_cast<int>(n_chunks), draft_tokens, cu_block, B, max_block, accept_len,
-      next_token, row_argmax, nullptr);
+      next_token, row_argmax, nullptr, B * max_block);
   e = cudaGetLastError();
   if (e != cudaSuccess) return fail(ORTHRUS_ERR_CUDA, "consensus launch: %s", cudaGetErrorString(e));
   return ok();
@@ -555,5 +556,171 @@ const char* orthrus_status_string(orthrus_status_t s) {
 const char* orthrus_last_error(void) { return g_last_error.c_str(); }
 
 int32_t orthrus_abi_version(void) { return ORTHRUS_ABI_VERSION; }
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// LM head + greedy token
+
+namespace {
+
+struct LmPlan {
+  int R, mt, N, n_m, n_n, n_tiles, stages, grid, box_a, box_b;
+  uint32_t stage_bytes, a_bytes;
+  size_t smem;
+};
+
+// Tile shape: with more than 128 rows two M=128 blocks share each w_head tile
+// (half the w_head reads per FLOP); N is the multiple of 16 in [128, 256] whose
+// tile count fills the SMs' waves best (time ~ waves * N), ties to the wider N.
+// With at most 128 rows (a memory-bound shape) one block per tile, N = 256, and
+// the accumulator is double buffered.
+orthrus_status_t plan_lm(int R, int d, int V, int sms, LmPlan* pl) {
+  if (R < 1 || d < 1 || V < 1) return fail(ORTHRUS_ERR_INVALID_ARG, "R %d, d %d, V %d", R, d, V);
+  if (d % kLmKStep)
+    return fail(ORTHRUS_ERR_UNSUPPORTED, "d_model = %d (a multiple of 64)", d);
+  pl->R = R;
+  pl->mt = R > 128 ? 2 : 1;
+  if (pl->mt == 1) {
+    pl->N = std::min(256, (V + 63) / 64 * 64);
+  } else {
+    int bestN = 256;
+    long long best = -1;
+    const long long n_m = (R + 255) / 256;
+    for (int N = 256; N >= 128; N -= 16) {
+      const long long tiles = n_m * ((V + N - 1) / N);
+      const long long cost = ((tiles + sms - 1) / sms) * N;
+      if (best < 0 || cost * 100 < best * 99) {
+        best = cost;
+        bestN = N;
+      }
+    }
+    pl->N = std::min(bestN, (V + 15) / 16 * 16);
+  }
+  pl->n_m = (R + 128 * pl->mt - 1) / (128 * pl->mt);
+  pl->n_n = (V + pl->N - 1) / pl->N;
+  const long long tiles = static_cast<long long>(pl->n_m) * pl->n_n;
+  if (tiles >= (1ll << 31)) return fail(ORTHRUS_ERR_UNSUPPORTED, "too many tiles");
+  pl->n_tiles = static_cast<int>(tiles);
+  pl->a_bytes = static_cast<uint32_t>(pl->mt) * kLmABlock;
+  pl->stage_bytes = pl->a_bytes + static_cast<uint32_t>(pl->N) * 128u;
+  const size_t budget = 232448;  // dynamic shared memory per CTA
+  const int st = static_cast<int>((budget - 1024 - LmLayout::kMiscBytes) / pl->stage_bytes);
+  pl->stages = std::min(st, kLmMaxStages);
+  if (pl->stages < 2) return fail(ORTHRUS_ERR_UNSUPPORTED, "tile does not fit shared memory");
+  pl->smem = lm_smem_bytes(pl->stages, pl->stage_bytes);
+  pl->grid = std::min(pl->n_tiles, std::max(sms, 1));
+  pl->box_a = std::min(128 * pl->mt, R);
+  pl->box_b = std::min(pl->N, V);
+  return ORTHRUS_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t orthrus_lm_head_workspace_size(int32_t total_rows) {
+  if (total_rows < 1) return 0;
+  return round_up(static_cast<size_t>(total_rows) * sizeof(unsigned long long), 256);
+}
+
+orthrus_status_t orthrus_lm_head_consensus(const void* hidden, const void* w_head,
+                                           int32_t d_model, int32_t V, int32_t total_rows,
+                                           const int32_t* draft_tokens, const int32_t* cu_block,
+                                           int32_t B, int32_t max_block, int32_t* accept_len,
+                                           int32_t* next_token, int32_t* row_argmax,
+                                           int32_t* prefix_lens, void* workspace,
+                                           size_t workspace_bytes, int32_t* error_flag,
+                                           void* stream) {
+  if (B < 0 || max_block < 1 || total_rows < 0)
+    return fail(ORTHRUS_ERR_INVALID_ARG, "B %d, max_block %d, total_rows %d", B, max_block,
+                total_rows);
+  const long long R64 = total_rows > 0 ? total_rows : static_cast<long long>(B) * max_block;
+  if (R64 >= (1ll << 31)) return fail(ORTHRUS_ERR_UNSUPPORTED, "too many rows");
+  if (!cu_block && R64 < static_cast<long long>(B) * max_block)
+    return fail(ORTHRUS_ERR_INVALID_ARG, "total_rows < B * max_block without cu_block");
+  LmPlan pl;
+  orthrus_status_t s = plan_lm(R64 > 0 ? static_cast<int>(R64) : 1, d_model, V, 148, &pl);
+  if (s != ORTHRUS_OK) return s;
+  if (B == 0) return ok();
+  if (!hidden || !w_head || !draft_tokens || !accept_len || !next_token || !workspace)
+    return fail(ORTHRUS_ERR_INVALID_ARG, "a required pointer is NULL");
+  if (!aligned(hidden, 16) || !aligned(w_head, 16) || !aligned(workspace, 16))
+    return fail(ORTHRUS_ERR_INVALID_ARG, "hidden, w_head and workspace must be 16-byte aligned");
+  const int R = static_cast<int>(R64);
+  if (workspace_bytes < orthrus_lm_head_workspace_size(R))
+    return fail(ORTHRUS_ERR_INVALID_ARG, "workspace %zu bytes < %zu needed", workspace_bytes,
+                orthrus_lm_head_workspace_size(R));
+  int sms = 0;
+  const int dev = device_sm_count(&sms);
+  if (dev < 0) return fail(ORTHRUS_ERR_CUDA, "no current CUDA device");
+  s = plan_lm(R, d_model, V, sms, &pl);
+  if (s != ORTHRUS_OK) return s;
+  static std::atomic<size_t> smem_set[kMaxDevices];
+  if (smem_set[dev].load() < pl.smem) {
+    cudaError_t e = cudaFuncSetAttribute(lm_head_argmax_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(pl.smem));
+    if (e != cudaSuccess)
+      return fail(ORTHRUS_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    smem_set[dev].store(pl.smem);
+  }
+  CUtensorMap ta, tb;
+  {
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(d_model), static_cast<cuuint64_t>(R)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(d_model) * 2};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(kLmKStep),
+                               static_cast<cuuint32_t>(pl.box_a)};
+    if (!make_map(&ta, hidden, 2, dims, strides, box))
+      return fail(ORTHRUS_ERR_CUDA, "tensor map for hidden");
+  }
+  {
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(d_model), static_cast<cuuint64_t>(V)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(d_model) * 2};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(kLmKStep),
+                               static_cast<cuuint32_t>(pl.box_b)};
+    if (!make_map(&tb, w_head, 2, dims, strides, box))
+      return fail(ORTHRUS_ERR_CUDA, "tensor map for w_head");
+  }
+  LmArgs a;
+  a.R = R;
+  a.V = V;
+  a.d = d_model;
+  a.N = pl.N;
+  a.mt = pl.mt;
+  a.n_m = pl.n_m;
+  a.n_tiles = pl.n_tiles;
+  a.k_steps = d_model / kLmKStep;
+  a.stages = pl.stages;
+  a.stage_bytes = pl.stage_bytes;
+  a.a_bytes = pl.a_bytes;
+  a.tx_bytes = static_cast<uint32_t>(pl.box_a + pl.box_b) * 128u;
+  a.idesc = idesc_bf16_f32(128, static_cast<uint32_t>(pl.N), 0);
+  a.keys = static_cast<unsigned long long*>(workspace);
+  a.error_flag = error_flag;
+  a.timeout_ns = wait_timeout_ns();
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(workspace, 0, static_cast<size_t>(R) * 8, st);
+  if (e != cudaSuccess) return fail(ORTHRUS_ERR_CUDA, "key reset: %s", cudaGetErrorString(e));
+  lm_head_argmax_kernel<<<pl.grid, kLmThreads, pl.smem, st>>>(ta, tb, a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(ORTHRUS_ERR_CUDA, "lm_head launch: %s", cudaGetErrorString(e));
+  const int warps = 8;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((B + warps - 1) / warps);
+  cfg.blockDim = dim3(warps * 32);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, consensus_finalize_kernel,
+                         static_cast<const unsigned long long*>(workspace), 1, draft_tokens,
+                         cu_block, static_cast<int>(B), static_cast<int>(max_block), accept_len,
+                         next_token, row_argmax, prefix_lens, R);
+  if (e != cudaSuccess) return fail(ORTHRUS_ERR_CUDA, "finalize launch: %s", cudaGetErrorString(e));
+  return ok();
+}
 
 }  // extern "C"

@@ -64,6 +64,11 @@ lib.orthrus_consensus_commit.argtypes = [_vp, _i64, _i32, _vp, _vp, _i32, _i32, 
 lib.orthrus_kv_append.restype = _i32
 lib.orthrus_kv_append.argtypes = [_vp, _vp, _vp, _i32, _vp, _vp, _i32, _vp, _i32, _i32, _vp, _vp,
                                   _i32, _i32, _i32, _i32, _vp, _vp]
+lib.orthrus_lm_head_workspace_size.restype = _sz
+lib.orthrus_lm_head_workspace_size.argtypes = [_i32]
+lib.orthrus_lm_head_consensus.restype = _i32
+lib.orthrus_lm_head_consensus.argtypes = [_vp, _vp, _i32, _i32, _i32, _vp, _vp, _i32, _i32, _vp, _vp,
+                                          _vp, _vp, _vp, _sz, _vp, _vp]
 lib.orthrus_consensus_noalloc.restype = _i32
 lib.orthrus_consensus_noalloc.argtypes = [_vp, _i64, _i32, _vp, _vp, _i32, _i32, _vp, _vp, _vp, _vp]
 lib.orthrus_status_string.restype = ctypes.c_char_p
@@ -237,6 +242,36 @@ def consensus_noalloc(verify_logits, draft_tokens, cu_block, B: int, max_block: 
                                        int(B), int(max_block), _ptr(accept_len), _ptr(next_token),
                                        _ptr(row_argmax), _stream(stream))
     _check(st, "orthrus_consensus_noalloc")
+
+
+def lm_head_workspace_size(total_rows: int) -> int:
+    return int(lib.orthrus_lm_head_workspace_size(int(total_rows)))
+
+
+def lm_head_consensus(hidden, w_head, draft_tokens, cu_block, B: int, max_block: int, accept_len,
+                      next_token, workspace, row_argmax=None, prefix_lens=None, error_flag=None,
+                      stream=None):
+    """``orthrus_lm_head_consensus``: greedy tokens of ``hidden @ w_head.T`` (never
+    materialised) and the consensus outputs, written in place."""
+    _need(hidden, "hidden", torch.bfloat16, 2)
+    _need(w_head, "w_head", torch.bfloat16, 2)
+    if hidden.shape[1] != w_head.shape[1]:
+        raise ValueError("hidden and w_head must share d_model")
+    _need(draft_tokens, "draft_tokens", torch.int32, 1)
+    _need(accept_len, "accept_len", torch.int32, 1)
+    _need(next_token, "next_token", torch.int32, 1)
+    _need(workspace, "workspace", torch.uint8)
+    for name, t in (("cu_block", cu_block), ("row_argmax", row_argmax),
+                    ("prefix_lens", prefix_lens), ("error_flag", error_flag)):
+        if t is not None:
+            _need(t, name, torch.int32)
+    st = lib.orthrus_lm_head_consensus(_ptr(hidden), _ptr(w_head), hidden.shape[1],
+                                       w_head.shape[0], hidden.shape[0], _ptr(draft_tokens),
+                                       _ptr(cu_block), int(B), int(max_block), _ptr(accept_len),
+                                       _ptr(next_token), _ptr(row_argmax), _ptr(prefix_lens),
+                                       _ptr(workspace), workspace.numel(), _ptr(error_flag),
+                                       _stream(stream))
+    _check(st, "orthrus_lm_head_consensus")
 
 
 def kv_append(k_block, v_block, cu_block, max_block: int, accept_len, prefix_lens, page_table,

@@ -221,6 +221,48 @@ ORTHRUS_API orthrus_status_t orthrus_consensus_commit(const float* verify_logits
                                                       size_t workspace_bytes, void* stream);
 
 /*
+ * Fused LM head + greedy consensus (technical summary §2.3 items 2-3 with §2.1:
+ * the frozen AR model scores every block row over the vocabulary, and its
+ * greedy token decides acceptance). For every block row r in [0, R):
+ *
+ *   t_r = argmax_v  sum_k hidden[r, k] * w_head[v, k]
+ *
+ * (bf16 products accumulated in fp32 by the tensor cores, in an unspecified
+ * order; ties go to the lowest v, NaN counts as -inf). The logits are never
+ * written: each vocabulary tile's row maxima are combined in the workspace.
+ * From the t_r, accept_len / next_token / row_argmax (and, when prefix_lens is
+ * given, the commit prefix_lens[b] += accept_len[b]) follow the rule of
+ * orthrus_consensus exactly.
+ *
+ *   hidden        device bf16 [R, d_model], row-major (the block rows' final
+ *                 hidden states), R = total_rows, or B * max_block when 0
+ *   w_head        device bf16 [V, d_model], row-major (one row per vocabulary
+ *                 entry: the output projection's [out, in] layout)
+ *   d_model       a multiple of 64
+ *   draft_tokens  device int32 [R]
+ *   cu_block      device int32 [B+1] or NULL (every K_b = max_block); a
+ *                 sequence whose rows fall outside [0, R) gets accept_len 0
+ *                 and next_token -1
+ *   accept_len, next_token  device int32 [B] (written)
+ *   row_argmax    device int32 [R] or NULL (written when given)
+ *   prefix_lens   device int32 [B] or NULL (advanced by accept_len when given)
+ *   workspace     device scratch of orthrus_lm_head_workspace_size(R) bytes,
+ *                 16-byte aligned; contents need no initialisation
+ *   error_flag    optional device int32: ORTHRUS_FLAG_TIMEOUT if a pipeline
+ *                 wait of the GEMM gave up (its rows' results are then invalid)
+ * Launches a 8*R-byte memset, the GEMM/argmax kernel (one CTA per SM) and the
+ * consensus finalize kernel. Errors: INVALID_ARG (null pointer, misalignment,
+ * short workspace, bad sizes), UNSUPPORTED (d_model not a multiple of 64, too
+ * many rows), CUDA.
+ */
+ORTHRUS_API size_t orthrus_lm_head_workspace_size(int32_t total_rows);
+ORTHRUS_API orthrus_status_t orthrus_lm_head_consensus(
+    const void* hidden, const void* w_head, int32_t d_model, int32_t V, int32_t total_rows,
+    const int32_t* draft_tokens, const int32_t* cu_block, int32_t B, int32_t max_block,
+    int32_t* accept_len, int32_t* next_token, int32_t* row_argmax, int32_t* prefix_lens,
+    void* workspace, size_t workspace_bytes, int32_t* error_flag, void* stream);
+
+/*
  * Commit (technical summary §2.3 item 3, commit the synchronised prefix and
  * truncate the cache; agents-report.net commentary, "core design", the accepted
  * tokens' KV appended to the shared cache). For every sequence b, accepted row
