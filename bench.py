@@ -40,6 +40,7 @@ from diffusion_draft_ar_b200 import workloads as W  # noqa: E402
 METRIC = "block-attn KV GB/s (% HBM roofline) at K=32; consensus rows/s; blocks/s"
 UNIT = "GB/s"
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 ATTN_SRC = os.path.join(ROOT, "diffusion_draft_ar_b200", "csrc", "block_attn.cuh")
 TRAFFIC_SUMMARY = os.path.join(ROOT, "profiles", "block_attn_qwen3_8b.md")
 
@@ -83,6 +84,66 @@ def peak_hbm():
         return v, "measured"
     except Exception:
         return FALLBACK_HBM_GBS, "fallback"
+
+
+def peak_bf16():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured cuBLAS bf16 burst"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def measure_lm_head(O, w: W.Workload, m: W.BatchMeta, dev, stream, calls: int = 20):
+    """The fused LM head + greedy consensus on the workload's verify rows (the
+    step before consensus when the logits are not materialised): hidden [R, d]
+    x w_head [V, d]^T, random bf16 operands of the model's shape. Timed alone,
+    CUDA events on the launching stream; w_head (> L2) is re-read every call."""
+    if w.d_model is None or w.vocab is None:
+        return None
+    R, d, V = m.R, w.d_model, w.vocab
+    hidden, w_head = W.lm_head_inputs(R, d, V, dev)
+    cu = m.cu_block.to(dev)
+    drafts = torch.zeros(R, dtype=torch.int32, device=dev)
+    acc = torch.zeros(m.B, dtype=torch.int32, device=dev)
+    nxt = torch.zeros(m.B, dtype=torch.int32, device=dev)
+    ws = torch.empty(O.lm_head_workspace_size(R), dtype=torch.uint8, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    sp = ctypes.c_void_p(stream.cuda_stream)
+    args = (hidden.data_ptr(), w_head.data_ptr(), d, V, R, drafts.data_ptr(), cu.data_ptr(), m.B,
+            w.max_block, acc.data_ptr(), nxt.data_ptr(), None, None, ws.data_ptr(), ws.numel(),
+            err.data_ptr(), sp)
+
+    def call():
+        st = O.lib.orthrus_lm_head_consensus(*args)
+        if st:
+            raise RuntimeError(f"orthrus_lm_head_consensus: {O.lib.orthrus_last_error().decode()}")
+
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(calls):
+        call()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if int(err.item()) != 0:
+        raise RuntimeError(f"lm_head device error flag {int(err.item())}")
+    us = e0.elapsed_time(e1) / calls * 1e3
+    flops = 2.0 * R * d * V
+    tflops = flops / (us * 1e-6) / 1e12
+    peak, src = peak_bf16()
+    del hidden, w_head
+    return {"workload": f"{w.name} verify rows through the LM head: {R} x {d} x {V} (bf16, fp32 acc)",
+            "us": us, "calls": calls, "tflops": tflops,
+            "w_head_gbs": 2.0 * V * d / (us * 1e-6) / 1e9,
+            "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak, "unit": "TFLOP/s",
+                         "frac": tflops / peak, "peak_source": src},
+            "kernels_per_call": 2, "note": "memset of the row keys, GEMM+argmax kernel, "
+                                           "consensus finalize; logits never written"}
 
 
 def traffic_per_launch():
@@ -410,6 +471,8 @@ def run_ours(args):
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / e2e_steps
     e2e_value = world * b_step / (e2e_ms * 1e-3) / 1e9
 
+    lm_head = None if args.no_lm_head else measure_lm_head(O, w, m, dev, stream)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, budget_s=args.cpu_seconds)
@@ -450,6 +513,7 @@ def run_ours(args):
                             "D2H of both outputs, accept lengths and next tokens; "
                             "the KV cache stays resident"},
             "gpu_launches": args.steps * launches_per_step,
+            "lm_head": lm_head,
             "clocks": clocks,
         }
         print(json.dumps(line), flush=True)
@@ -468,6 +532,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-lm-head", action="store_true",
+                    help="skip the separate fused LM-head measurement")
     ap.add_argument("--commit", choices=["write", "append"], default="write",
                     help="write: VERIFY attention stores the block K/V and consensus advances "
                          "the lengths (write-then-truncate); append: separate kv_append launch")

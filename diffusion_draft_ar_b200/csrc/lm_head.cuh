@@ -24,15 +24,19 @@
 // time and the second read hits L2.
 //
 // Roles (320 threads, one CTA per SM):
-//   warp 0      TMA producer (one lane): A box (mt*128 rows x 64) and B box
-//               (N rows x 64) per K step into a ring of stages.
+//   warp 0      TMA producer, two lanes: per K step lane 0 arms the stage's
+//               barrier and issues the A box (mt*128 rows x 64), lane 1 the B
+//               box (N rows x 64). A box issue holds its thread for a few
+//               hundred cycles whatever the box size, so one issuing thread
+//               capped the ring at about one stage per microsecond; two lanes
+//               issue side by side.
 //   warp 1      MMA issuer: mt x 4 tcgen05.mma (M=128, N, K=16) per stage into
 //               TMEM; commits release the stage and, after a tile's last step,
 //               publish the accumulator. Owns the TMEM allocation.
 //   warps 2-9   epilogue, two groups of four warps (each group covers the four
 //               TMEM lane quarters): with mt = 2 group g reduces accumulator g
 //               (rows g*128 + lane); with mt = 1 the two groups split the
-//               columns of the one accumulator. Each thread scans its row's
+//               columns of the one accumulator (at a multiple of 32). Each thread scans its row's
 //               columns in increasing order (strict >, so ties keep the lower
 //               index and NaN never wins) and atomically maxes its key.
 // With mt = 1 the accumulator is double buffered (two 256-column slots), so
@@ -144,7 +148,12 @@ __global__ void __launch_bounds__(kLmThreads, 1)
   const int n_slots = a.mt == 1 ? 2 : 1;
 
   if (warp == kLmProducerWarp) {
-    if (lane == 0) {
+    if (lane < 2) {
+      // Both lanes walk every stage in order (each waits on every phase of
+      // every empty barrier, so a parity wait is never two phases ahead).
+      // Lane 1's bytes may land before lane 0 arms the barrier: the
+      // transaction count goes negative for a moment, and the phase cannot
+      // complete before lane 0's arrival.
       int s = 0;
       uint32_t ph = 0;
       long long issued = 0;
@@ -154,9 +163,12 @@ __global__ void __launch_bounds__(kLmThreads, 1)
         for (int ks = 0; ks < a.k_steps; ++ks) {
           if (!wait(bar(LmLayout::empty(s)), ph ^ 1u)) { ok = false; break; }
           const uint32_t st = base + s * a.stage_bytes;
-          mbar_arrive_expect_tx(bar(LmLayout::full(s)), a.tx_bytes);
-          tma_load_2d(st, &tm_a, bar(LmLayout::full(s)), ks * kLmKStep, m * 128 * a.mt);
-          tma_load_2d(st + a.a_bytes, &tm_b, bar(LmLayout::full(s)), ks * kLmKStep, n * a.N);
+          if (lane == 0) {
+            mbar_arrive_expect_tx(bar(LmLayout::full(s)), a.tx_bytes);
+            tma_load_2d(st, &tm_a, bar(LmLayout::full(s)), ks * kLmKStep, m * 128 * a.mt);
+          } else {
+            tma_load_2d(st + a.a_bytes, &tm_b, bar(LmLayout::full(s)), ks * kLmKStep, n * a.N);
+          }
           ++issued;
           if (++s == a.stages) { s = 0; ph ^= 1u; }
         }
@@ -235,8 +247,11 @@ __global__ void __launch_bounds__(kLmThreads, 1)
         row = m * 256 + g * 128 + q * 32 + lane;
         col = 256u * static_cast<uint32_t>(g);
       } else {
-        c0 = g * (a.N >> 1);
-        c1 = c0 + (a.N >> 1);
+        // the two groups split the columns at a multiple of 32 (TMEM loads
+        // start on 32-column boundaries)
+        const int split = ((a.N >> 1) + 31) & ~31;
+        c0 = g == 0 ? 0 : split;
+        c1 = g == 0 ? split : a.N;
         row = m * 128 + q * 32 + lane;
         col = 256u * static_cast<uint32_t>(slot);
       }
@@ -245,7 +260,23 @@ __global__ void __launch_bounds__(kLmThreads, 1)
       const int c_end = min(c1, a.V - v0);
       float best = -__int_as_float(0x7f800000);
       int bidx = -1;
-      for (int c = c0; c < c1; c += 32) {  // c0, c1: multiples of 16, warp-uniform
+      int c = c0;
+      if (c_end >= c1) {
+        // whole slice inside the vocabulary: 64 columns per TMEM wait, no bounds test
+        for (; c + 64 <= c1; c += 64) {
+          float x0[32], x1[32];
+          tmem_ld32(tmem + lane_addr + col + c, x0);
+          tmem_ld32(tmem + lane_addr + col + c + 32, x1);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            if (x0[e] > best) { best = x0[e]; bidx = v0 + c + e; }
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            if (x1[e] > best) { best = x1[e]; bidx = v0 + c + 32 + e; }
+        }
+      }
+      for (; c < c1; c += 32) {  // c, c1: multiples of 16, warp-uniform
         float x0[16], x1[16];
         const bool two = c + 16 < c1;
         tmem_ld16(tmem + lane_addr + col + c, x0);

@@ -571,10 +571,16 @@ struct LmPlan {
 };
 
 // Tile shape: with more than 128 rows two M=128 blocks share each w_head tile
-// (half the w_head reads per FLOP); N is the multiple of 16 in [128, 256] whose
-// tile count fills the SMs' waves best (time ~ waves * N), ties to the wider N.
-// With at most 128 rows (a memory-bound shape) one block per tile, N = 256, and
-// the accumulator is double buffered.
+// (half the w_head reads per FLOP) and N = 256, the widest MMA. Measured on the
+// Qwen3-8B head (512 x 4096 x 151936): an MMA inside this loop costs about the
+// same whatever N (shared-memory port traffic of the TMA writes and operand
+// reads, not the tensor core, sets the pace), so the widest tile beats a
+// narrower one that would fill the last wave better (600 us at N = 256, 670 at
+// 208, 730 at 192). With at most 128 rows the head is memory-bound (one block
+// per tile, the accumulator double buffered): a tile's time follows its w_head
+// bytes, so N (a multiple of 32 in [128, 256], the two epilogue groups taking
+// half each) minimises waves x N; at V = 151936 that is 224 (679 tiles, 4.6
+// waves) rather than 256 (594 tiles: 4 full waves and 2 tiles).
 orthrus_status_t plan_lm(int R, int d, int V, int sms, LmPlan* pl) {
   if (R < 1 || d < 1 || V < 1) return fail(ORTHRUS_ERR_INVALID_ARG, "R %d, d %d, V %d", R, d, V);
   if (d % kLmKStep)
@@ -583,19 +589,18 @@ orthrus_status_t plan_lm(int R, int d, int V, int sms, LmPlan* pl) {
   pl->mt = R > 128 ? 2 : 1;
   if (pl->mt == 1) {
     pl->N = std::min(256, (V + 63) / 64 * 64);
-  } else {
-    int bestN = 256;
-    long long best = -1;
-    const long long n_m = (R + 255) / 256;
-    for (int N = 256; N >= 128; N -= 16) {
-      const long long tiles = n_m * ((V + N - 1) / N);
-      const long long cost = ((tiles + sms - 1) / sms) * N;
-      if (best < 0 || cost * 100 < best * 99) {
-        best = cost;
-        bestN = N;
+    if (V > 256) {
+      long long best = -1;
+      for (int N = 256; N >= 128; N -= 32) {
+        const long long waves = ((V + N - 1) / N + sms - 1) / sms;
+        if (best < 0 || waves * N < best) {
+          best = waves * N;
+          pl->N = N;
+        }
       }
     }
-    pl->N = std::min(bestN, (V + 15) / 16 * 16);
+  } else {
+    pl->N = std::min(256, (V + 15) / 16 * 16);
   }
   pl->n_m = (R + 128 * pl->mt - 1) / (128 * pl->mt);
   pl->n_n = (V + pl->N - 1) / pl->N;

@@ -57,6 +57,7 @@ class Workload:
     rounds: int = 1
     headroom: int = 0                        # append slots reserved per sequence
     kv_split_tokens: int = 0                 # 0: library-chosen split
+    d_model: int | None = None               # hidden size feeding the LM head (Qwen3 config)
 
     @property
     def G(self) -> int:
@@ -75,10 +76,10 @@ WORKLOADS: dict[str, Workload] = {
                      vocab=512, logit_std=1.0, p_match=0.7, headroom=8),
     "qwen3_1p7b": Workload("qwen3_1p7b", B=1, Hq=16, Hkv=8, D=128, prefix_len=4096, block=32,
                            paged=False, vocab=VOCAB_QWEN3, logit_std=2.0, p_match=0.8,
-                           headroom=32),
+                           headroom=32, d_model=2048),
     "qwen3_8b": Workload("qwen3_8b", B=16, Hq=32, Hkv=8, D=128, prefix_len=8192, block=32,
                          paged=True, vocab=VOCAB_QWEN3, logit_std=1.0, p_match=0.8,
-                         headroom=32),
+                         headroom=32, d_model=4096),
     "longctx": Workload("longctx", B=1, Hq=32, Hkv=8, D=128, prefix_len=131072, block=32,
                         paged=True, views=("verify",), vocab=None, headroom=32,
                         kv_split_tokens=2048),
@@ -272,7 +273,18 @@ def ceil_div(a: int, b: int) -> int:
 
 
 __all__ = [
-    "Workload", "WORKLOADS", "BatchMeta", "make_meta", "WorkloadInputs", "RoundInputs",
+    "lm_head_inputs", "Workload", "WORKLOADS", "BatchMeta", "make_meta", "WorkloadInputs", "RoundInputs",
     "drafts_from_targets", "randn_bf16", "randn_f32", "cache_bytes_per_token",
     "bf16_bits", "sentinel_fill_", "ceil_div", "VIEW_NAMES", "VOCAB_QWEN3",
 ]
+
+
+def lm_head_inputs(R: int, d_model: int, V: int, device, seed: int = 0):
+    """Seeded synthetic LM-head operands: final hidden states N(0, 1) [R, d] and an
+    output projection N(0, 1/d) [V, d] (so each score is about N(0, 1)), both
+    bf16, drawn on ``device``. Random weights of the shape only: no checkpoint."""
+    g = torch.Generator(device=device)
+    g.manual_seed(seed + 7)
+    hidden = randn_bf16((R, d_model), g, device)
+    w = randn_bf16((V, d_model), g, device, std=d_model ** -0.5)
+    return hidden, w
