@@ -203,12 +203,27 @@ __global__ void __launch_bounds__(kLmThreads, 1)
         if (!wait(bar(LmLayout::full(s)), ph)) { ok = false; break; }
         tc_fence_after();
         const uint32_t st = base + s * a.stage_bytes;
+        // Both loops have compile-time bounds: with a run-time bound around
+        // elect.sync + tcgen05.mma each issue cost ~200 cycles (the tensor core
+        // starved at ~1600 cycles per K step whatever N); unrolled, the issue
+        // runs ahead of the tensor core.
+        if (a.mt == 2) {
 #pragma unroll
-        for (int kk = 0; kk < kLmKStep / 16; ++kk) {
-          const uint64_t bd = smem_desc_sw128(st + a.a_bytes + kk * 32, 16, 1024);
-          for (int j = 0; j < a.mt; ++j) {
-            const uint64_t ad = smem_desc_sw128(st + j * kLmABlock + kk * 32, 16, 1024);
-            const uint32_t acc = tmem + 256u * static_cast<uint32_t>(a.mt == 2 ? j : slot);
+          for (int kk = 0; kk < kLmKStep / 16; ++kk) {
+            const uint64_t bd = smem_desc_sw128(st + a.a_bytes + kk * 32, 16, 1024);
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+              const uint64_t ad = smem_desc_sw128(st + j * kLmABlock + kk * 32, 16, 1024);
+              if (elect_one())
+                mma_bf16_ss(tmem + 256u * j, ad, bd, a.idesc, (ks | kk) ? 1u : 0u);
+            }
+          }
+        } else {
+          const uint32_t acc = tmem + 256u * static_cast<uint32_t>(slot);
+#pragma unroll
+          for (int kk = 0; kk < kLmKStep / 16; ++kk) {
+            const uint64_t bd = smem_desc_sw128(st + a.a_bytes + kk * 32, 16, 1024);
+            const uint64_t ad = smem_desc_sw128(st + kk * 32, 16, 1024);
             if (elect_one()) mma_bf16_ss(acc, ad, bd, a.idesc, (ks | kk) ? 1u : 0u);
           }
         }
