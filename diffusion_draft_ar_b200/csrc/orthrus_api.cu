@@ -571,12 +571,11 @@ struct LmPlan {
 };
 
 // Tile shape: with more than 128 rows two M=128 blocks share each w_head tile
-// (half the w_head reads per FLOP) and N = 256, the widest MMA. Measured on the
-// Qwen3-8B head (512 x 4096 x 151936): an MMA inside this loop costs about the
-// same whatever N (shared-memory port traffic of the TMA writes and operand
-// reads, not the tensor core, sets the pace), so the widest tile beats a
-// narrower one that would fill the last wave better (600 us at N = 256, 670 at
-// 208, 730 at 192). With at most 128 rows the head is memory-bound (one block
+// (half the w_head reads per FLOP) and N = 192, the widest tile whose stage
+// (32 KB of hidden rows + N x 128 B of w_head) still fits four ring stages.
+// Measured on the Qwen3-8B head (512 x 4096 x 151936): 449 us at N = 192
+// (4 stages), 460 at 176, 463 at 256 and 466 at 208 (3 stages), 480 at 192
+// held to 3 stages. With at most 128 rows the head is memory-bound (one block
 // per tile, the accumulator double buffered): a tile's time follows its w_head
 // bytes, so N (a multiple of 32 in [128, 256], the two epilogue groups taking
 // half each) minimises waves x N; at V = 151936 that is 224 (679 tiles, 4.6
@@ -600,7 +599,7 @@ orthrus_status_t plan_lm(int R, int d, int V, int sms, LmPlan* pl) {
       }
     }
   } else {
-    pl->N = std::min(256, (V + 15) / 16 * 16);
+    pl->N = std::min(192, (V + 15) / 16 * 16);
   }
   pl->n_m = (R + 128 * pl->mt - 1) / (128 * pl->mt);
   pl->n_n = (V + pl->N - 1) / pl->N;
