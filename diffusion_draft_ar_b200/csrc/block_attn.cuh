@@ -74,9 +74,10 @@ struct AttnArgs {
   float scale_log2;  // softmax scale * log2(e)
   int q_box_rows;    // tokens per Q box: min(max_block, total_rows)
   int blk_box_rows;  // rows per block-K/V box: min(64, total_rows)
-  int chunked;       // 0: balanced ranges over num_ctas CTAs; 1: fixed chunks
-  int chunk_tiles;   // chunked: prefix tiles per chunk
-  int max_chunks;    // chunked: chunks per unit (grid = B * Hkv * max_chunks)
+  int chunked;       // 0: balanced ranges over num_ctas CTAs; 1: fixed chunks;
+                     // 2: proportional chunks (see prop_ctas)
+  int chunk_tiles;   // chunked == 1: prefix tiles per chunk
+  int max_chunks;    // chunked == 1: chunks per unit (grid = B * Hkv * max_chunks)
   int num_ctas;      // grid size
   unsigned long long timeout_ns;
   int fault_inject;  // test hook: 1 drops each CTA's first V copy (a wait must time out)
@@ -131,6 +132,18 @@ __device__ __forceinline__ int unit_chunks(const AttnArgs& a, int nt) {
 
 __device__ __forceinline__ long long range_begin(long long T, int c, int C) {
   return T * c / C;
+}
+
+// Proportional chunks (few long units): of the C CTAs, a unit with nt tiles
+// gets 1 + floor((C - U) * nt / T), at most nt, where U counts the units with
+// tiles and T sums their tiles (so the counts add up to at most C); chunk k of
+// c covers the unit's tiles [k*nt/c, (k+1)*nt/c). Units stay whole inside a
+// CTA, and equal lengths get equal chunks. Sequence b's units take the CTAs
+// after those of sequences 0..b-1, head by head.
+__device__ __forceinline__ int prop_ctas(long long T, int U, int C, int nt) {
+  if (nt <= 0) return 0;
+  const long long c = 1 + (long long)(C - U) * nt / T;
+  return c < nt ? (int)c : nt;
 }
 
 // What the schedule needs of sequence b: tiles, clamped prefix length, K_b and
@@ -333,7 +346,31 @@ __device__ __forceinline__ bool schedule_prologue(const AttnArgs& a, uint8_t* sm
   }
   const long long T = block_sum_ll(part, scan);  // also publishes the table
 
-  if (a.chunked) {
+  if (a.chunked == 2) {
+    if (tid == 0) {
+      int U = 0;
+      for (int bb = 0; bb < a.B; ++bb) U += tab.nt(a, bb) > 0 ? a.Hkv : 0;
+      int b = a.B, h = 0, t = 0;
+      long long rem = 0, base = 0;
+      for (int bb = 0; bb < a.B && U > 0; ++bb) {
+        const int nt = tab.nt(a, bb);
+        const int c = prop_ctas(T, U, a.num_ctas, nt);
+        const long long span = (long long)a.Hkv * c;
+        if (blockIdx.x < base + span) {
+          const int off = (int)(blockIdx.x - base);
+          const int k = off % c;
+          b = bb;
+          h = off / c;
+          t = (int)((long long)k * nt / c);
+          rem = (long long)(k + 1) * nt / c - t;
+          break;
+        }
+        base += span;
+      }
+      sc[0] = b, sc[1] = h, sc[2] = t;
+      *srem = rem;
+    }
+  } else if (a.chunked) {
     if (tid == 0) {
       int b = a.B, h = 0, t = 0;
       long long rem = 0;
@@ -1143,7 +1180,29 @@ __global__ void __launch_bounds__(kCombineThreads)
   if (warp == 0) {
     int skip = 0, count = 0, c_lo = 0;
     long long T = 0, s_u = 0;
-    if (a.chunked) {
+    if (a.chunked == 2) {
+      // the attention kernel's allocation: T, U, then the CTAs of sequences < b
+      long long t_part = 0;
+      int u_part = 0;
+      for (int bb = lane; bb < a.B; bb += 32) {
+        const int n = seq_tiles(a, bb);
+        t_part += (long long)a.Hkv * n;
+        u_part += n > 0 ? a.Hkv : 0;
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        t_part += __shfl_xor_sync(0xffffffffu, t_part, o);
+        u_part += __shfl_xor_sync(0xffffffffu, u_part, o);
+      }
+      long long before = 0;
+      for (int bb = lane; bb < b; bb += 32)
+        before += (long long)a.Hkv * prop_ctas(t_part, u_part, a.num_ctas, seq_tiles(a, bb));
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) before += __shfl_xor_sync(0xffffffffu, before, o);
+      count = prop_ctas(t_part, u_part, a.num_ctas, nt);
+      c_lo = (int)(before + (long long)h * count);  // first part (= CTA) of this unit
+      skip = count <= 1;
+    } else if (a.chunked) {
       count = unit_chunks(a, nt);
       skip = count <= 1;
     } else {
@@ -1180,6 +1239,10 @@ __global__ void __launch_bounds__(kCombineThreads)
   const int c_lo = sh_clo, count = sh_count;
 
   auto part_of = [&](int k, bool& use) -> int {
+    if (a.chunked == 2) {
+      use = true;
+      return c_lo + k;
+    }
     if (a.chunked) {
       use = true;
       return u * a.max_chunks + k;

@@ -171,6 +171,17 @@ orthrus_status_t plan_attn(const orthrus_attn_params* p, int sms, AttnPlan* pl) 
     pl->grid = p->B * p->Hkv;
     pl->parts = pl->grid;
     pl->combine = false;
+  } else if (p->max_ctas == 0 && static_cast<long long>(p->B) * p->Hkv < (3LL * sms) / 4) {
+    // Few units (long contexts): every unit gets a share of the SMs in
+    // proportion to its tiles, cut into near-equal chunks on the device from
+    // the actual lengths. No CTA switches units, which the balanced ranges
+    // below do whenever a range boundary falls inside a unit.
+    pl->chunked = 2;
+    pl->chunk_tiles = 0;
+    pl->max_chunks = 0;
+    pl->grid = std::max(sms, 1);
+    pl->parts = pl->grid;
+    pl->combine = true;
   } else {
     pl->chunked = 0;
     pl->chunk_tiles = 0;

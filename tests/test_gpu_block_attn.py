@@ -134,6 +134,21 @@ def test_prefix_beyond_page_table_is_flagged():
 
 
 @pytest.mark.parametrize("view", VIEWS)
+def test_few_long_units_proportional_chunks(view):
+    """Few units of very different lengths (prefixes of 0, 3000 and 40000 tokens,
+    2 KV heads): the default schedule gives every unit SMs in proportion to its
+    tiles, cut into near-equal chunks, and merges them; every output checked,
+    and the same outputs with an explicit balanced split."""
+    w = small_workload(name="few_long", B=3, Hq=8, Hkv=2, D=128, page_size=64, prefix_len=None,
+                       prefix_range=(40000, 40000), block=None, block_choices=(32,), paged=True,
+                       headroom=64)
+    wi = W.WorkloadInputs(w, seed=4)
+    wi.meta.prefix_lens[:] = torch.tensor([0, 3000, 40000], dtype=torch.int32)
+    _full_parity(wi, view)
+    _full_parity(wi, view, max_ctas=148)
+
+
+@pytest.mark.parametrize("view", VIEWS)
 def test_qwen3_8b_sampled(view):
     """Qwen3-8B-shaped layer (16 x L=8192, K=32, 32/8 heads, random pages) in the
     launch configuration the bench times; sampled outputs against the oracle."""
