@@ -76,6 +76,7 @@ struct LmArgs {
   unsigned long long* keys;  // [R] packed (value, index) keys, zeroed before the launch
   int* error_flag;
   unsigned long long timeout_ns;
+  int fault_inject;   // test hook: 1 drops each CTA's first w_head copy (a wait must time out)
 };
 
 struct LmLayout {
@@ -166,7 +167,7 @@ __global__ void __launch_bounds__(kLmThreads, 1)
           if (lane == 0) {
             mbar_arrive_expect_tx(bar(LmLayout::full(s)), a.tx_bytes);
             tma_load_2d(st, &tm_a, bar(LmLayout::full(s)), ks * kLmKStep, m * 128 * a.mt);
-          } else {
+          } else if (!(a.fault_inject == 1 && issued == 0)) {
             tma_load_2d(st + a.a_bytes, &tm_b, bar(LmLayout::full(s)), ks * kLmKStep, n * a.N);
           }
           ++issued;

@@ -714,6 +714,11 @@ orthrus_status_t orthrus_lm_head_consensus(const void* hidden, const void* w_hea
   a.keys = static_cast<unsigned long long*>(workspace);
   a.error_flag = error_flag;
   a.timeout_ns = wait_timeout_ns();
+  {
+    // the attention call's test hook: ORTHRUS_FAULT_INJECT=1 withholds one copy per CTA
+    const char* fi = std::getenv("ORTHRUS_FAULT_INJECT");
+    a.fault_inject = fi ? std::atoi(fi) : 0;
+  }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e = cudaMemsetAsync(workspace, 0, static_cast<size_t>(R) * 8, st);
   if (e != cudaSuccess) return fail(ORTHRUS_ERR_CUDA, "key reset: %s", cudaGetErrorString(e));

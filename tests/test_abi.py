@@ -188,3 +188,26 @@ def test_consensus_commit_rejects_bad_arguments(O, args, status):
                                         a["max_block"], a["acc"], a["nxt"], a["am"], a["lens"],
                                         a["workspace"], a["workspace_bytes"], None)
     assert st == status
+
+
+@pytest.mark.parametrize("args,status", [
+    (dict(d=96), 2), (dict(d=0), 1), (dict(V=0), 1), (dict(B=-1), 1), (dict(max_block=0), 1),
+    (dict(hidden=None), 1), (dict(w_head=None), 1), (dict(draft=None), 1), (dict(ws=None), 1),
+    (dict(hidden=0x10008), 1), (dict(ws_bytes=8), 1), (dict(total_rows=4, cu=None), 1),
+])
+def test_lm_head_rejects_bad_arguments(O, args, status):
+    a = dict(hidden=0x10000, w_head=0x20000, d=128, V=1000, total_rows=0, draft=0x30000,
+             cu=0x40000, B=2, max_block=8, acc=0x50000, nxt=0x60000, ws=0x70000,
+             ws_bytes=1 << 20)
+    a.update(args)
+    st = O.lib.orthrus_lm_head_consensus(a["hidden"], a["w_head"], a["d"], a["V"], a["total_rows"],
+                                         a["draft"], a["cu"], a["B"], a["max_block"], a["acc"],
+                                         a["nxt"], None, None, a["ws"], a["ws_bytes"], None, None)
+    assert st == status
+    assert O.lib.orthrus_last_error() != b""
+
+
+def test_lm_head_workspace_size(O):
+    assert O.lm_head_workspace_size(512) == 4096
+    assert O.lm_head_workspace_size(33) == 512
+    assert O.lm_head_workspace_size(0) == 0

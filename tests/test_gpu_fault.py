@@ -55,3 +55,48 @@ def test_withheld_copy_times_out_and_context_survives():
                        capture_output=True, text=True, timeout=300)
     assert r.returncode == 0, r.stdout + r.stderr
     assert "FAULT-OK" in r.stdout
+
+
+CHILD_LM = r"""
+import os, sys, numpy as np, torch
+sys.path.insert(0, ROOT)
+import oracle
+from diffusion_draft_ar_b200 import workloads as W
+from diffusion_draft_ar_b200 import orthrus as O
+g = torch.Generator().manual_seed(2)
+R, d, V = 96, 128, 5000
+hidden = torch.randint(-1, 2, (R, d), generator=g).to(torch.bfloat16)
+w_head = torch.randint(-2, 3, (V, d), generator=g).to(torch.bfloat16)
+cu = torch.tensor([0, 32, 64, 96], dtype=torch.int32)
+drafts = torch.randint(0, V, (R,), generator=g, dtype=torch.int32)
+acc = torch.zeros(3, dtype=torch.int32, device="cuda")
+nxt = torch.zeros(3, dtype=torch.int32, device="cuda")
+am = torch.zeros(R, dtype=torch.int32, device="cuda")
+ws = torch.empty(O.lm_head_workspace_size(R), dtype=torch.uint8, device="cuda")
+err = torch.zeros(1, dtype=torch.int32, device="cuda")
+args = (hidden.cuda(), w_head.cuda(), drafts.cuda(), cu.cuda(), 3, 32, acc, nxt, ws)
+os.environ["ORTHRUS_FAULT_INJECT"] = "1"
+O.lm_head_consensus(*args, row_argmax=am, error_flag=err)
+torch.cuda.synchronize()
+flag = int(err.item())
+assert flag & O.FLAG_TIMEOUT, flag
+os.environ["ORTHRUS_FAULT_INJECT"] = "0"
+err.zero_()
+O.lm_head_consensus(*args, row_argmax=am, error_flag=err)
+torch.cuda.synchronize()
+assert int(err.item()) == 0
+t = oracle.greedy_tokens(oracle.lm_head_logits(W.bf16_bits(hidden), W.bf16_bits(w_head)))
+assert am.cpu().numpy().tolist() == t.tolist()
+print("FAULT-OK", flag)
+"""
+
+
+def test_lm_head_withheld_copy_times_out_and_context_survives():
+    """The fused LM head's pipeline waits are bounded the same way: a withheld
+    w_head copy makes the MMA warp's wait run out; the call reports
+    ORTHRUS_FLAG_TIMEOUT, every role winds down, and the next call is exact."""
+    env = dict(os.environ, ORTHRUS_WAIT_TIMEOUT_MS="50", PYTHONPATH=ROOT)
+    r = subprocess.run([sys.executable, "-c", "ROOT = %r\n" % ROOT + CHILD_LM], env=env,
+                       capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stdout + r.stderr
+    assert "FAULT-OK" in r.stdout
