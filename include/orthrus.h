@@ -6,7 +6,7 @@
  * anchor plus K-1 mask slots) over the KV cache that a frozen autoregressive
  * (AR) view built, then has the AR view verify the whole block in one pass and
  * keeps the drafts that equal the AR greedy tokens. This library implements the
- * three data-parallel steps of one round:
+ * data-parallel steps of one round:
  *
  *   orthrus_block_attn  attention of the block rows over the shared paged prefix
  *                       cache plus the block's own K/V, in the DIFFUSION view
@@ -14,7 +14,15 @@
  *                       (causal inside the block);
  *   orthrus_consensus   greedy argmax of the verify logits and the left-to-right
  *                       exact match against the drafts;
- *   orthrus_kv_append   commit: write the accepted rows' K/V into the cache.
+ *   orthrus_kv_append   commit: write the accepted rows' K/V into the cache;
+ * and fused forms of them:
+ *   orthrus_block_attn_verify_write + orthrus_consensus_commit
+ *                       write-then-truncate: the VERIFY attention stores the
+ *                       whole block's K/V, consensus advances the lengths;
+ *   orthrus_lm_head_consensus
+ *                       the AR model's LM head (hidden states x output
+ *                       projection) with the greedy argmax in its epilogue,
+ *                       then the consensus rule; the logits are never written.
  *
  * Conventions shared by every call:
  *   - Every pointer marked "device" is a device pointer owned by the caller; the
