@@ -654,8 +654,12 @@ orthrus_status_t orthrus_lm_head_consensus(const void* hidden, const void* w_hea
   if (R64 >= (1ll << 31)) return fail(ORTHRUS_ERR_UNSUPPORTED, "too many rows");
   if (!cu_block && R64 < static_cast<long long>(B) * max_block)
     return fail(ORTHRUS_ERR_INVALID_ARG, "total_rows < B * max_block without cu_block");
+  // Shape checks first, with a nominal SM count: no CUDA call before the
+  // arguments are known to be valid. The real count only sizes the grid.
+  constexpr int kNominalSms = 148;
   LmPlan pl;
-  orthrus_status_t s = plan_lm(R64 > 0 ? static_cast<int>(R64) : 1, d_model, V, 148, &pl);
+  orthrus_status_t s =
+      plan_lm(R64 > 0 ? static_cast<int>(R64) : 1, d_model, V, kNominalSms, &pl);
   if (s != ORTHRUS_OK) return s;
   if (B == 0) return ok();
   if (!hidden || !w_head || !draft_tokens || !accept_len || !next_token || !workspace)
