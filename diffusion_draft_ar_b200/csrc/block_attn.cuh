@@ -140,10 +140,12 @@ __device__ __forceinline__ long long range_begin(long long T, int c, int C) {
 // c covers the unit's tiles [k*nt/c, (k+1)*nt/c). Units stay whole inside a
 // CTA, and equal lengths get equal chunks. Sequence b's units take the CTAs
 // after those of sequences 0..b-1, head by head.
+constexpr int kMinChunkTiles = 4;  // a split pays a partial and the combine
 __device__ __forceinline__ int prop_ctas(long long T, int U, int C, int nt) {
   if (nt <= 0) return 0;
   const long long c = 1 + (long long)(C - U) * nt / T;
-  return c < nt ? (int)c : nt;
+  const int cap = nt / kMinChunkTiles > 1 ? nt / kMinChunkTiles : 1;
+  return c < cap ? (int)c : cap;
 }
 
 // What the schedule needs of sequence b: tiles, clamped prefix length, K_b and

@@ -176,12 +176,17 @@ orthrus_status_t plan_attn(const orthrus_attn_params* p, int sms, AttnPlan* pl) 
     // proportion to its tiles, cut into near-equal chunks on the device from
     // the actual lengths. No CTA switches units, which the balanced ranges
     // below do whenever a range boundary falls inside a unit.
+    // A chunk is at least kMinChunkTiles tiles (a split pays a partial and
+    // the combine); when no unit can be that long, each stays whole in one CTA
+    // and the combine kernel is not launched.
+    const long long max_nt = (max_tokens + kTileN - 1) / kTileN + 1;
+    const bool whole = max_nt / kMinChunkTiles <= 1;
     pl->chunked = 2;
     pl->chunk_tiles = 0;
     pl->max_chunks = 0;
-    pl->grid = std::max(sms, 1);
+    pl->grid = whole ? p->B * p->Hkv : std::max(sms, 1);
     pl->parts = pl->grid;
-    pl->combine = true;
+    pl->combine = !whole;
   } else {
     pl->chunked = 0;
     pl->chunk_tiles = 0;
