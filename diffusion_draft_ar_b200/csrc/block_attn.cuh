@@ -1131,7 +1131,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   } else if (warp < kSoftmaxWarp0) {
     mma_role<D>(a, smem, tmem, abort_flag, warp - kMmaWarp0, tab, start);
   } else if (warp == kWriterWarp) {
-    if (a.write_block) block_writer_role<D>(a, tab, start);
+    if (a.write_block) {
+      // Start the copies once this CTA's first K tile has landed, off the
+      // pipeline's cold start (VERIFY minus DIFFUSION time per call: 1.5 us
+      // with the copies at kernel start, 0.7 us from here). The wait is
+      // bounded like every other; it gives up only if the pipeline stalled.
+      mbar_wait(smem_u32(smem) + Lay::kBarOff + 8u * Lay::kBarKFull, 0, abort_flag,
+                a.timeout_ns);
+      block_writer_role<D>(a, tab, start);
+    }
   } else {
     softmax_role<D>(a, smem, tmem, abort_flag, tab, start);
   }
