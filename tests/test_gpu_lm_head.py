@@ -191,3 +191,22 @@ def test_qwen3_8b_verify_rows_sampled():
         acc, nxt = oracle.accept_from_tokens(tb, drafts.numpy()[32 * b:32 * b + 32],
                                              np.array([0, 32], np.int32))
         assert got["acc"][b] == acc[0] and got["nxt"][b] == nxt[0]
+
+
+@pytest.mark.parametrize("R,d,V", [(1, 64, 257), (7, 192, 17), (129, 64, 1000), (255, 128, 513),
+                                   (257, 64, 300), (130, 192, 4097)])
+def test_edge_tilings_integer_exact(R, d, V):
+    """Ragged tilings on exact (integer) scores: one row; a second 128-row block
+    holding a single row (R = 129); row and vocabulary tails of one element
+    (R = 257, V = 257, 4097); d_model of three K steps. Every token, accept
+    length and next token must equal the oracle's."""
+    hidden, w, _, drafts = make_case(R, d, V, seed=R * 7 + V, integer=True)
+    cuts = sorted({0, R, *[min(R, x) for x in (1, R // 3, R // 2)]})
+    cu = torch.tensor(cuts, dtype=torch.int32)
+    K = int((cu[1:] - cu[:-1]).max())
+    got = run_gpu(hidden, w, cu, drafts, K)
+    t = oracle.greedy_tokens(oracle.lm_head_logits(bits(hidden), bits(w)))
+    np.testing.assert_array_equal(got["am"], t)
+    acc, nxt = oracle.accept_from_tokens(t, drafts.numpy(), cu.numpy())
+    np.testing.assert_array_equal(got["acc"], acc)
+    np.testing.assert_array_equal(got["nxt"], nxt)
