@@ -18,7 +18,6 @@ from __future__ import annotations
 
 import argparse
 import ctypes
-import datetime
 import hashlib
 import json
 import os
@@ -35,6 +34,7 @@ if ROOT not in sys.path:
 import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
+from diffusion_draft_ar_b200 import dist as D  # noqa: E402
 from diffusion_draft_ar_b200 import workloads as W  # noqa: E402
 
 METRIC = "block-attn KV GB/s (% HBM roofline) at K=32; consensus rows/s; blocks/s"
@@ -205,35 +205,6 @@ class ClockSampler:
                 "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
 
 
-def dist_setup():
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                device_id=torch.device("cuda", local))
-    else:
-        torch.cuda.set_device(0)
-    return world, rank, local
-
-
-def barrier(world):
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
-
-
-def max_over_ranks(x: float, world: int) -> float:
-    if world == 1:
-        return x
-    import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
-
-
 # ---------------------------------------------------------------------------
 # CPU oracle on a bounded sample (reference arm and cpu_baseline)
 
@@ -326,11 +297,11 @@ def run_reference(args):
 # GPU arm
 
 def run_ours(args):
-    world, rank, local = dist_setup()
+    world, rank, local = D.init("nccl", timeout_s=300)
     from diffusion_draft_ar_b200 import orthrus as O
     w = W.WORKLOADS[args.workload]
     dev = torch.device("cuda", torch.cuda.current_device())
-    wi = W.WorkloadInputs(w, device=dev, seed=rank)
+    wi = W.WorkloadInputs(w, device=dev, seed=D.rank_seed(0, rank))
     m, r = wi.meta, wi.rounds[0]
     stream = torch.cuda.current_stream()
     lens0 = m.prefix_lens.to(dev)
@@ -413,18 +384,18 @@ def run_ours(args):
     sampler = ClockSampler(dev.index)
     sampler.start()
     time.sleep(0.3)  # let the sampler take its first reading
-    barrier(world)
+    D.barrier(world)
     torch.cuda.synchronize()
     t_start.record(stream)
     for i in range(args.steps):
         step(evs[i])
     t_end.record(stream)
     torch.cuda.synchronize()
-    barrier(world)
+    D.barrier(world)
     clocks = sampler.stop()
     total_ms = t_start.elapsed_time(t_end)
     part = np.array([[e[j].elapsed_time(e[j + 1]) for j in range(4)] for e in evs])  # ms
-    total_ms = max_over_ranks(total_ms, world)
+    total_ms = D.max_over_ranks(total_ms, world)
     ms_step = total_ms / args.steps
     t_diff, t_ver, t_cons, t_app = (float(x) for x in part.mean(0))
 
@@ -456,7 +427,7 @@ def run_ours(args):
     d2h = sum(t.numel() * t.element_size() for t in h_out.values())
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    barrier(world)
+    D.barrier(world)
     torch.cuda.synchronize()
     e0.record(stream)
     for _ in range(e2e_steps):
@@ -467,8 +438,8 @@ def run_ours(args):
             h_out[k].copy_(d_out[k], non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
-    barrier(world)
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / e2e_steps
+    D.barrier(world)
+    e2e_ms = D.max_over_ranks(e0.elapsed_time(e1), world) / e2e_steps
     e2e_value = world * b_step / (e2e_ms * 1e-3) / 1e9
 
     lm_head = None if args.no_lm_head else measure_lm_head(O, w, m, dev, stream)
@@ -526,9 +497,7 @@ def run_ours(args):
             "clocks": clocks,
         }
         print(json.dumps(line), flush=True)
-    if world > 1:
-        import torch.distributed as dist
-        dist.destroy_process_group()
+    D.finish(world)
 
 
 def main():
