@@ -2,6 +2,7 @@
 // before any CUDA call), TMA descriptor encoding, launch configuration.
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <algorithm>
 #include <atomic>
@@ -42,6 +43,29 @@ orthrus_status_t ok() {
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// NVTX range named after the C-ABI call, in the "orthrus" domain, around the
+// host side of each call (argument checks and launches). NVTX v3 forwards to
+// a profiler only when one is attached; otherwise a push/pop is a predicted
+// branch on an unset function pointer.
+nvtxDomainHandle_t nvtx_domain() {
+  static nvtxDomainHandle_t d = nvtxDomainCreateA("orthrus");
+  return d;
+}
+
+struct NvtxRange {
+  explicit NvtxRange(const char* name) {
+    nvtxEventAttributes_t ev = {};
+    ev.version = NVTX_VERSION;
+    ev.size = NVTX_EVENT_ATTRIB_STRUCT_SIZE;
+    ev.messageType = NVTX_MESSAGE_TYPE_ASCII;
+    ev.message.ascii = name;
+    nvtxDomainRangePushEx(nvtx_domain(), &ev);
+  }
+  ~NvtxRange() { nvtxDomainRangePop(nvtx_domain()); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
+
 constexpr int kMaxDevices = 64;
 
 int device_sm_count(int* sms) {
@@ -56,6 +80,29 @@ int device_sm_count(int* sms) {
   }
   *sms = v;
   return dev;
+}
+
+// Failure-detection test hook. ORTHRUS_FAULT_INJECT=n, read once per process,
+// makes the first n attention or LM-head launches of the process withhold one
+// copy per CTA, so that a bounded pipeline wait runs out; every later launch
+// is normal. Only a test's child process sets it. A process without it pays
+// one load of a cached counter per launch and no getenv.
+std::atomic<int>& fault_inject_budget() {
+  static std::atomic<int> v([] {
+    const char* e = std::getenv("ORTHRUS_FAULT_INJECT");
+    const int n = e ? std::atoi(e) : 0;
+    return n > 0 ? n : 0;
+  }());
+  return v;
+}
+
+int fault_inject_mode() {
+  std::atomic<int>& b = fault_inject_budget();
+  int n = b.load(std::memory_order_relaxed);
+  while (n > 0) {
+    if (b.compare_exchange_weak(n, n - 1, std::memory_order_relaxed)) return 1;
+  }
+  return 0;
 }
 
 unsigned long long wait_timeout_ns() {
@@ -272,12 +319,7 @@ orthrus_status_t launch_attn(const orthrus_attn_params* p, const AttnPlan& pl, i
   a.max_chunks = pl.max_chunks;
   a.num_ctas = pl.grid;
   a.timeout_ns = wait_timeout_ns();
-  {
-    // Test hook for failure detection, read on every call: ORTHRUS_FAULT_INJECT=1
-    // withholds one copy per CTA so that a pipeline wait runs out.
-    const char* fi = std::getenv("ORTHRUS_FAULT_INJECT");
-    a.fault_inject = fi ? std::atoi(fi) : 0;
-  }
+  a.fault_inject = fault_inject_mode();
   a.out_v8 = aligned(p->out, 32) ? 1 : 0;
   a.write_block = write_block ? 1 : 0;
   a.kb_rows = static_cast<const uint4*>(p->k_block);
@@ -371,10 +413,12 @@ static orthrus_status_t block_attn_entry(const orthrus_attn_params* p, void* str
 }
 
 orthrus_status_t orthrus_block_attn(const orthrus_attn_params* p, void* stream) {
+  NvtxRange r("orthrus_block_attn");
   return block_attn_entry(p, stream, false);
 }
 
 orthrus_status_t orthrus_block_attn_verify_write(const orthrus_attn_params* p, void* stream) {
+  NvtxRange r("orthrus_block_attn_verify_write");
   if (p && p->view != ORTHRUS_VIEW_VERIFY)
     return fail(ORTHRUS_ERR_INVALID_ARG, "write-then-truncate needs the VERIFY view");
   return block_attn_entry(p, stream, true);
@@ -439,6 +483,7 @@ orthrus_status_t orthrus_consensus(const float* verify_logits, int64_t ld, int32
                                    int32_t B, int32_t max_block, int32_t* accept_len,
                                    int32_t* next_token, int32_t* row_argmax, void* workspace,
                                    size_t workspace_bytes, void* stream) {
+  NvtxRange r("orthrus_consensus");
   return consensus_entry(verify_logits, ld, V, draft_tokens, cu_block, B, max_block, accept_len,
                          next_token, row_argmax, nullptr, workspace, workspace_bytes, stream);
 }
@@ -449,6 +494,7 @@ orthrus_status_t orthrus_consensus_commit(const float* verify_logits, int64_t ld
                                           int32_t* next_token, int32_t* row_argmax,
                                           int32_t* prefix_lens, void* workspace,
                                           size_t workspace_bytes, void* stream) {
+  NvtxRange r("orthrus_consensus_commit");
   if (B > 0 && !prefix_lens) return fail(ORTHRUS_ERR_INVALID_ARG, "prefix_lens is NULL");
   return consensus_entry(verify_logits, ld, V, draft_tokens, cu_block, B, max_block, accept_len,
                          next_token, row_argmax, prefix_lens, workspace, workspace_bytes, stream);
@@ -461,6 +507,7 @@ orthrus_status_t orthrus_kv_append(const void* k_block, const void* v_block,
                                    int32_t max_pages_per_seq, int32_t num_pages, void* k_cache,
                                    void* v_cache, int32_t B, int32_t Hkv, int32_t D,
                                    int32_t page_size, int32_t* error_flag, void* stream) {
+  NvtxRange r("orthrus_kv_append");
   if (B < 0 || Hkv < 1 || D < 8 || D % 8 || page_size < 1 || max_pages_per_seq < 0 ||
       num_pages < 0 || (!cu_block && max_block < 1))
     return fail(ORTHRUS_ERR_INVALID_ARG, "bad sizes (B %d, Hkv %d, D %d, P %d)", B, Hkv, D,
@@ -495,22 +542,15 @@ static __device__ __align__(256) unsigned long long g_consensus_scratch[kNoAlloc
 
 namespace {
 
-// Device address of g_consensus_scratch on the current device. In host code
-// the array's name is only a host-side stand-in, so the address is looked up
-// once per device (with that device current) and cached.
-unsigned long long* noalloc_scratch(int* dev_out) {
-  static std::mutex mu;
-  static void* addr[kMaxDevices];
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  *dev_out = dev;
-  std::lock_guard<std::mutex> lock(mu);
-  if (!addr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_consensus_scratch) != cudaSuccess || !p) return nullptr;
-    addr[dev] = p;
-  }
-  return static_cast<unsigned long long*>(addr[dev]);
+// Device address of g_consensus_scratch in the current device's context. In
+// host code the array's name is only a host-side stand-in, so the address is
+// looked up with that device current. It is looked up on every call (a symbol
+// lookup in the loaded module, no allocation): a cached address would go
+// stale if the context were reset and the module loaded again elsewhere.
+unsigned long long* noalloc_scratch() {
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_consensus_scratch) != cudaSuccess || !p) return nullptr;
+  return static_cast<unsigned long long*>(p);
 }
 
 }  // namespace
@@ -522,6 +562,7 @@ orthrus_status_t orthrus_consensus_noalloc(const float* verify_logits, int64_t l
                                            int32_t B, int32_t max_block, int32_t* accept_len,
                                            int32_t* next_token, int32_t* row_argmax,
                                            void* stream) {
+  NvtxRange r("orthrus_consensus_noalloc");
   if (B < 0) return fail(ORTHRUS_ERR_INVALID_ARG, "B = %d < 0", B);
   if (V < 1 || ld < V) return fail(ORTHRUS_ERR_INVALID_ARG, "V = %d, ld = %lld", V, (long long)ld);
   if (max_block < 1) return fail(ORTHRUS_ERR_INVALID_ARG, "max_block = %d", max_block);
@@ -538,8 +579,7 @@ orthrus_status_t orthrus_consensus_noalloc(const float* verify_logits, int64_t l
                 "request needs %lld scratch keys (B*max_block*ceil(V/16384)); the built-in "
                 "array holds %lld",
                 keys, kNoAllocScratchKeys);
-  int dev = 0;
-  unsigned long long* part = noalloc_scratch(&dev);
+  unsigned long long* part = noalloc_scratch();
   if (!part) return fail(ORTHRUS_ERR_CUDA, "cannot resolve the scratch array's device address");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   dim3 grid(static_cast<unsigned>(n_chunks), static_cast<unsigned>(R_max));
@@ -570,6 +610,12 @@ const char* orthrus_status_string(orthrus_status_t s) {
 }
 
 const char* orthrus_last_error(void) { return g_last_error.c_str(); }
+
+orthrus_status_t orthrus_status_from_flags(int32_t flags) {
+  if (flags == 0) return ORTHRUS_OK;
+  if (flags & ORTHRUS_FLAG_TIMEOUT) return ORTHRUS_ERR_TIMEOUT;
+  return ORTHRUS_ERR_DEVICE_CHECK;
+}
 
 int32_t orthrus_abi_version(void) { return ORTHRUS_ABI_VERSION; }
 
@@ -652,6 +698,7 @@ orthrus_status_t orthrus_lm_head_consensus(const void* hidden, const void* w_hea
                                            int32_t* prefix_lens, void* workspace,
                                            size_t workspace_bytes, int32_t* error_flag,
                                            void* stream) {
+  NvtxRange r("orthrus_lm_head_consensus");
   if (B < 0 || max_block < 1 || total_rows < 0)
     return fail(ORTHRUS_ERR_INVALID_ARG, "B %d, max_block %d, total_rows %d", B, max_block,
                 total_rows);
@@ -723,11 +770,7 @@ orthrus_status_t orthrus_lm_head_consensus(const void* hidden, const void* w_hea
   a.keys = static_cast<unsigned long long*>(workspace);
   a.error_flag = error_flag;
   a.timeout_ns = wait_timeout_ns();
-  {
-    // the attention call's test hook: ORTHRUS_FAULT_INJECT=1 withholds one copy per CTA
-    const char* fi = std::getenv("ORTHRUS_FAULT_INJECT");
-    a.fault_inject = fi ? std::atoi(fi) : 0;
-  }
+  a.fault_inject = fault_inject_mode();
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e = cudaMemsetAsync(workspace, 0, static_cast<size_t>(R) * 8, st);
   if (e != cudaSuccess) return fail(ORTHRUS_ERR_CUDA, "key reset: %s", cudaGetErrorString(e));

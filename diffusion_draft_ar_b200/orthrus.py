@@ -77,6 +77,8 @@ lib.orthrus_last_error.restype = ctypes.c_char_p
 lib.orthrus_last_error.argtypes = []
 lib.orthrus_abi_version.restype = _i32
 lib.orthrus_abi_version.argtypes = []
+lib.orthrus_status_from_flags.restype = _i32
+lib.orthrus_status_from_flags.argtypes = [_i32]
 
 
 class OrthrusError(RuntimeError):

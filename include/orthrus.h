@@ -41,6 +41,9 @@
  *   - bf16 is IEEE binary32's upper 16 bits; all layouts are row-major and
  *     densely packed.
  *   - Outputs must not alias inputs.
+ *   - Each compute call pushes an NVTX range named after itself in the
+ *     "orthrus" domain around its host-side work (checks and launches); the
+ *     range costs nothing measurable unless a profiler is attached.
  */
 #ifndef ORTHRUS_H_
 #define ORTHRUS_H_
@@ -65,9 +68,14 @@ typedef enum {
   ORTHRUS_ERR_INVALID_ARG = 1,  /* a pointer, size or layout argument is wrong */
   ORTHRUS_ERR_UNSUPPORTED = 2,  /* valid, but outside what the kernels implement */
   ORTHRUS_ERR_CUDA = 3,         /* the CUDA runtime refused a launch or query */
-  ORTHRUS_ERR_TIMEOUT = 4,      /* reserved for callers mapping ORTHRUS_FLAG_TIMEOUT */
-  ORTHRUS_ERR_DEVICE_CHECK = 5  /* reserved for callers mapping the other flag bits */
+  ORTHRUS_ERR_TIMEOUT = 4,      /* a pipeline wait gave up (orthrus_status_from_flags) */
+  ORTHRUS_ERR_DEVICE_CHECK = 5  /* a device-side data check failed (orthrus_status_from_flags) */
 } orthrus_status_t;
+/* The launch calls return only OK, INVALID_ARG, UNSUPPORTED or CUDA: they are
+ * asynchronous, so what the kernels find (ORTHRUS_FLAG_* bits in the caller's
+ * error_flag word) is known only once the stream has reached that point.
+ * orthrus_status_from_flags turns such a word, read by the caller after a
+ * stream synchronisation, into TIMEOUT or DEVICE_CHECK. */
 
 /* Bits OR-ed into *error_flag by the kernels. */
 #define ORTHRUS_FLAG_BAD_PAGE 0x1   /* a page_table entry was outside [0, num_pages) */
@@ -318,9 +326,13 @@ ORTHRUS_API orthrus_status_t orthrus_kv_append(const void* k_block, const void* 
  *   - the request must fit: B * max_block * ceil(V / 16384) <= 65536 (for
  *     V = 151936 that is B * max_block <= 6553 rows); larger requests return
  *     ORTHRUS_ERR_UNSUPPORTED and launch nothing;
- *   - the first call on a device looks up the array's device address for that
- *     device (a runtime symbol query, no allocation); make that first call
- *     before any stream capture;
+ *   - every call looks up the array's address in the current device's
+ *     context (a runtime symbol lookup, no allocation);
+ *   - the array is reserved when the library's device code is loaded on a
+ *     device, which under CUDA's lazy module loading can be the first call of
+ *     this library there: a caller that reserves nearly all of HBM should make
+ *     one library call on each device at start-up, before that reservation,
+ *     and also before any stream capture;
  *   - every call on a device uses the same array, so calls whose kernels can
  *     overlap on the GPU (different streams without ordering) race: order them
  *     on one stream or with events. Nothing in the array needs to start at
@@ -337,6 +349,13 @@ ORTHRUS_API orthrus_status_t orthrus_consensus_noalloc(const float* verify_logit
 
 /* Static description of a status code. */
 ORTHRUS_API const char* orthrus_status_string(orthrus_status_t status);
+
+/* Status for a word of ORTHRUS_FLAG_* bits that the kernels OR-ed into a
+ * caller's error_flag (read by the caller after synchronising the stream):
+ * ORTHRUS_OK for 0, ORTHRUS_ERR_TIMEOUT when ORTHRUS_FLAG_TIMEOUT is set (that
+ * CTA's results are missing), ORTHRUS_ERR_DEVICE_CHECK for any other bit (bad
+ * page ids or lengths: the flagged work was skipped). Host only; no CUDA call. */
+ORTHRUS_API orthrus_status_t orthrus_status_from_flags(int32_t flags);
 
 /* Detail of the last failed call on this host thread ("" when none). */
 ORTHRUS_API const char* orthrus_last_error(void);

@@ -335,12 +335,6 @@ static void argmax_row(void* ctx, int64_t r) {
   a->row_argmax[r] = idx;
 }
 
-/* For each sequence b with block rows row0 .. row0+K_b-1:
- *   t_r  = greedy token of row r
- *   m_b  = number of leading rows whose draft equals t_r
- *   n_b  = min(m_b + 1, K_b)     (accepted drafts plus the AR correction)
- *   next = t_{row0 + n_b - 1}    (the token that becomes the next anchor)
- * A sequence with K_b = 0 gets n_b = 0 and next = -1. row_argmax may be NULL. */
 /* For each sequence b with block rows row0 .. row0+K_b-1 and greedy tokens t:
  *   m_b  = number of leading rows whose draft equals t_r
  *   n_b  = min(m_b + 1, K_b)     (accepted drafts plus the AR correction)

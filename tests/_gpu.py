@@ -65,6 +65,8 @@ def oracle_args_dev(wi: W.WorkloadInputs, view: str, round_idx: int = 0):
 
 
 def assert_attn_close(got_bf16: torch.Tensor, ref: np.ndarray, what: str = ""):
+    """Whole-tensor comparison: max |err| and relative RMS over every compared
+    output, the worst (row, head) reported."""
     got = got_bf16.detach().to("cpu").double().numpy()
     assert got.shape == ref.shape, (got.shape, ref.shape)
     assert np.isfinite(got).all(), f"{what}: non-finite output"
@@ -72,6 +74,8 @@ def assert_attn_close(got_bf16: torch.Tensor, ref: np.ndarray, what: str = ""):
     den = np.sqrt(np.sum(ref * ref))
     rel = float(np.sqrt(np.sum(err * err)) / (den if den > 0 else 1.0))
     worst = np.unravel_index(int(np.argmax(err)), err.shape)
+    print(f"[parity] {what}: {err.size} outputs, max |err| {err.max():.3e} at {worst}, "
+          f"relative RMS {rel:.3e}")
     assert err.max() <= ATOL, f"{what}: max |err| {err.max():.3e} at {worst}"
     assert rel <= RTOL_RMS, f"{what}: relative RMS {rel:.3e}"
     return float(err.max()), rel

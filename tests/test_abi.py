@@ -50,6 +50,27 @@ def test_abi_version_and_status_strings(O):
     assert O.lib.orthrus_status_string(99) == b"unknown status"
 
 
+def test_status_from_flags(O):
+    f = O.lib.orthrus_status_from_flags
+    assert f(0) == O.OK
+    assert f(O.FLAG_TIMEOUT) == O.ERR_TIMEOUT
+    assert f(O.FLAG_TIMEOUT | O.FLAG_BAD_PAGE) == O.ERR_TIMEOUT
+    assert f(O.FLAG_BAD_PAGE) == O.ERR_DEVICE_CHECK
+    assert f(O.FLAG_BAD_LENGTH) == O.ERR_DEVICE_CHECK
+
+
+def test_noalloc_rejects_requests_beyond_its_array_on_the_host(O):
+    """The no-allocation consensus refuses a request whose keys exceed its fixed
+    array before any CUDA call (so this runs without a GPU)."""
+    V = 151936
+    B, K = 300, 32      # 9600 rows x 10 chunks = 96000 keys > 65536
+    st = O.lib.orthrus_consensus_noalloc(ctypes.c_void_p(16), V, V, ctypes.c_void_p(16), None,
+                                         B, K, ctypes.c_void_p(16), ctypes.c_void_p(16), None,
+                                         None)
+    assert st == O.ERR_UNSUPPORTED
+    assert b"scratch" in O.lib.orthrus_last_error()
+
+
 def test_param_struct_layout_matches_header(O):
     fields = [f[0] for f in O.AttnParams._fields_]
     prog = ["#include <stdio.h>", "#include <stddef.h>", '#include "orthrus.h"', "int main(void){",

@@ -8,7 +8,7 @@ import torch
 
 import oracle
 from diffusion_draft_ar_b200 import workloads as W
-from tests._gpu import DevAttn, assert_attn_close, gpu, lib, needs_cuda, sample_pairs
+from tests._gpu import DevAttn, assert_attn_close, gpu, lib, needs_cuda
 from tests._helpers import oracle_attn_args, small_workload
 
 pytestmark = [gpu, needs_cuda]
@@ -149,37 +149,87 @@ def test_few_long_units_proportional_chunks(view):
 
 
 @pytest.mark.parametrize("view", VIEWS)
-def test_qwen3_8b_sampled(view):
+def test_qwen3_8b_full(view):
     """Qwen3-8B-shaped layer (16 x L=8192, K=32, 32/8 heads, random pages) in the
-    launch configuration the bench times; sampled outputs against the oracle."""
+    launch configuration the bench times; every one of the 512 x 32 x 128 outputs
+    against the oracle."""
     wi = W.WorkloadInputs(W.WORKLOADS["qwen3_8b"], seed=0, device="cuda")
-    d = DevAttn(wi)
-    out = d.run(view)
-    assert int(d.err.item()) == 0
-    rows, heads = sample_pairs(wi.meta, wi.w.Hq, 192, seed=10)
-    ref = oracle.block_attn(*oracle_attn_args(wi, view), sel=(rows, heads))
-    got = out[torch.from_numpy(rows).cuda(), torch.from_numpy(heads).long().cuda()]
-    assert_attn_close(got, ref, f"qwen3_8b/{view}")
-    assert torch.isfinite(out.float()).all()
+    _full_parity(wi, view)
 
 
 @pytest.mark.parametrize("split", [2048, 0])
-def test_longctx_sampled(split):
-    """L = 131072, VERIFY view, split over 2048-token chunks (and balanced)."""
+def test_longctx_full(split):
+    """L = 131072, VERIFY view, split over 2048-token chunks (and the library's
+    proportional chunks); every output against the oracle."""
     wi = W.WorkloadInputs(W.WORKLOADS["longctx"], seed=0, device="cuda")
+    _full_parity(wi, "verify", kv_split=split)
+
+
+def _bias_block_keys(wi, score: float = 8.0, seed: int = 21):
+    """Every query of both views is the same direction u (|q| = 4) and every block
+    key is a multiple of u whose score is `score` + N(0, 1), so each block key
+    outweighs a prefix key (score ~ N(0, 0.35^2) at D = 128) by about e^8: a wrong
+    in-block mask moves outputs by O(1) even behind an 8192-token prefix."""
+    w = wi.w
+    r = wi.rounds[0]
+    g = torch.Generator().manual_seed(seed)
+    u = torch.randn(w.D, generator=g, dtype=torch.float64)
+    u = u / u.norm()
+    s = 1.0 / np.sqrt(w.D)
+    q = (4.0 * u).to(torch.bfloat16)
+    z = torch.randn(r.k_block["verify"].shape[:2], generator=g, dtype=torch.float64)
+    alpha = (score + z) / (s * 4.0)
+    kb = (alpha[..., None] * u).to(torch.bfloat16)
+    dev = r.q["verify"].device
+    for view in VIEWS:
+        r.q[view].copy_(q.to(dev).expand_as(r.q[view]))
+        r.k_block[view].copy_(kb.to(dev))
+        r.v_block[view].copy_(r.v_block["verify"])
+    return wi
+
+
+def test_qwen3_8b_block_bias_mask_sensitivity():
+    """Qwen3-8B-shaped layer with block keys scored +8 above the prefix: both views
+    match the oracle over every output, and they differ on every row but each
+    sequence's last (where the causal row sees the whole block), by O(1) on rows
+    that see at most half the block."""
+    wi = _bias_block_keys(W.WorkloadInputs(W.WORKLOADS["qwen3_8b"], seed=0, device="cuda"))
     d = DevAttn(wi)
-    out = d.run("verify", kv_split=split)
-    assert int(d.err.item()) == 0
-    rows, heads = sample_pairs(wi.meta, wi.w.Hq, 64, seed=11)
-    ref = oracle.block_attn(*oracle_attn_args(wi, "verify"), sel=(rows, heads))
-    got = out[torch.from_numpy(rows).cuda(), torch.from_numpy(heads).long().cuda()]
-    assert_attn_close(got, ref, f"longctx/{split}")
-    assert torch.isfinite(out.float()).all()
+    outs = {}
+    for view in VIEWS:
+        out = d.run(view)
+        ref = oracle.block_attn(*oracle_attn_args(wi, view))
+        assert int(d.err.item()) == 0
+        assert_attn_close(out, ref, f"qwen3_8b block bias/{view}")
+        outs[view] = out.float().cpu().numpy()
+    diff = np.abs(outs["diffusion"] - outs["verify"]).max(axis=(1, 2))  # per block row
+    K = wi.w.block
+    for b in range(wi.meta.B):
+        rows = diff[b * K:(b + 1) * K]
+        assert rows[:K // 2].min() > 0.1, (b, rows[:K // 2].min())  # at most half the block seen
+        assert rows[:K - 1].min() > 0.0, (b, rows[:K - 1].min())
+        assert rows[K - 1] == 0.0
 
 
 def test_views_differ_and_are_deterministic():
+    """Same inputs through both views: the DIFFUSION and VERIFY outputs differ on
+    every block row but each sequence's last (identical there), and a repeated
+    call is bit-identical."""
     wi = _ragged(seed=12)
     d = DevAttn(wi)
-    a = d.run("verify", max_ctas=5).clone()
-    b = d.run("verify", max_ctas=5).clone()
+    r = wi.rounds[0]
+    same = dict(q=r.q["verify"], kb=r.k_block["verify"], vb=r.v_block["verify"])
+    a = d.run("verify", max_ctas=5, **same).clone()
+    b = d.run("verify", max_ctas=5, **same).clone()
     assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    c = d.run("diffusion", max_ctas=5, **same).clone()
+    cu = wi.meta.cu_block.tolist()
+    for s in range(wi.meta.B):
+        r0, r1 = cu[s], cu[s + 1]
+        if r1 - r0 == 0:
+            continue
+        last_a, last_c = a[r1 - 1], c[r1 - 1]
+        assert torch.equal(last_a.view(torch.int16), last_c.view(torch.int16)), s
+        if r1 - r0 > 1:
+            dd = (a[r0:r1 - 1].float() - c[r0:r1 - 1].float()).abs().amax(dim=(1, 2))
+            assert (dd > 0).all(), (s, dd)

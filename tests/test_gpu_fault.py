@@ -1,8 +1,9 @@
 """Failure detection without a GPU fault: a copy the pipeline needs is withheld
-(ORTHRUS_FAULT_INJECT=1), so a bounded wait runs out; the kernel must report
-ORTHRUS_FLAG_TIMEOUT through the error word, return, and leave the CUDA context
-usable for the next, correct call. Runs in a child process so the short wait
-limit (ORTHRUS_WAIT_TIMEOUT_MS, read once per process) stays local to it."""
+(ORTHRUS_FAULT_INJECT=1: the first launch of the process withholds one copy per
+CTA), so a bounded wait runs out; the kernel must report ORTHRUS_FLAG_TIMEOUT
+through the error word, return, and leave the CUDA context usable for the
+next, correct call. Runs in a child process so the hook and the short wait
+limit (both read once per process) stay local to it."""
 import os
 import subprocess
 import sys
@@ -32,12 +33,11 @@ out = torch.zeros_like(args[0])
 err = torch.zeros(1, dtype=torch.int32, device="cuda")
 p = O.attn_params("verify", *args, out, w.max_block, max_ctas=4)
 ws = torch.empty(O.block_attn_workspace_size(p), dtype=torch.uint8, device="cuda")
-os.environ["ORTHRUS_FAULT_INJECT"] = "1"
 O.block_attn("verify", *args, out, ws, w.max_block, max_ctas=4, error_flag=err)
 torch.cuda.synchronize()
 flag = int(err.item())
 assert flag & O.FLAG_TIMEOUT, flag
-os.environ["ORTHRUS_FAULT_INJECT"] = "0"
+assert O.lib.orthrus_status_from_flags(flag) == O.ERR_TIMEOUT
 err.zero_()
 O.block_attn("verify", *args, out, ws, w.max_block, max_ctas=4, error_flag=err)
 torch.cuda.synchronize()
@@ -50,7 +50,8 @@ print("FAULT-OK", flag)
 
 
 def test_withheld_copy_times_out_and_context_survives():
-    env = dict(os.environ, ORTHRUS_WAIT_TIMEOUT_MS="50", PYTHONPATH=ROOT)
+    env = dict(os.environ, ORTHRUS_WAIT_TIMEOUT_MS="50", ORTHRUS_FAULT_INJECT="1",
+               PYTHONPATH=ROOT)
     r = subprocess.run([sys.executable, "-c", "ROOT = %r\n" % ROOT + CHILD], env=env,
                        capture_output=True, text=True, timeout=300)
     assert r.returncode == 0, r.stdout + r.stderr
@@ -75,12 +76,10 @@ am = torch.zeros(R, dtype=torch.int32, device="cuda")
 ws = torch.empty(O.lm_head_workspace_size(R), dtype=torch.uint8, device="cuda")
 err = torch.zeros(1, dtype=torch.int32, device="cuda")
 args = (hidden.cuda(), w_head.cuda(), drafts.cuda(), cu.cuda(), 3, 32, acc, nxt, ws)
-os.environ["ORTHRUS_FAULT_INJECT"] = "1"
 O.lm_head_consensus(*args, row_argmax=am, error_flag=err)
 torch.cuda.synchronize()
 flag = int(err.item())
 assert flag & O.FLAG_TIMEOUT, flag
-os.environ["ORTHRUS_FAULT_INJECT"] = "0"
 err.zero_()
 O.lm_head_consensus(*args, row_argmax=am, error_flag=err)
 torch.cuda.synchronize()
@@ -95,7 +94,8 @@ def test_lm_head_withheld_copy_times_out_and_context_survives():
     """The fused LM head's pipeline waits are bounded the same way: a withheld
     w_head copy makes the MMA warp's wait run out; the call reports
     ORTHRUS_FLAG_TIMEOUT, every role winds down, and the next call is exact."""
-    env = dict(os.environ, ORTHRUS_WAIT_TIMEOUT_MS="50", PYTHONPATH=ROOT)
+    env = dict(os.environ, ORTHRUS_WAIT_TIMEOUT_MS="50", ORTHRUS_FAULT_INJECT="1",
+               PYTHONPATH=ROOT)
     r = subprocess.run([sys.executable, "-c", "ROOT = %r\n" % ROOT + CHILD_LM], env=env,
                        capture_output=True, text=True, timeout=300)
     assert r.returncode == 0, r.stdout + r.stderr
