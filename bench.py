@@ -2,12 +2,22 @@
 """Throughput of one Orthrus block-decoding round on B200.
 
 A step is one pass of the whole hot path over one batch:
-  block attention (DIFFUSION view) -> block attention (VERIFY view)
-  -> greedy consensus over the verify logits -> KV append of the accepted rows
+  block attention (DIFFUSION view) -> block attention (VERIFY view, storing
+  the block K/V: write-then-truncate) -> greedy consensus over the verify
+  logits, which commits the accepted lengths
 on the Qwen3-8B-shaped workload (16 sequences, prefix 8192, block 32, 32/8
 heads, head dim 128, 64-token pages in a random permutation, vocabulary 151936),
-inputs resident in HBM. prefix_lens is restored (64-byte device copy) at the
-start of every step so each step appends at the same positions.
+inputs resident in HBM. L2 is scrubbed before every timed call (a 256 MB write
+then a 256 MB read of another buffer, outside the timed interval), so each call
+starts with none of its inputs in L2 and no dirty line to write back; the step
+time is the sum of the calls' event-timed intervals. prefix_lens is restored
+(64-byte device copy) at the start of every step so each step appends at the
+same positions.
+
+The same JSON line carries, measured the same way: the separate kv_append
+launch on this workload, the other workloads (Qwen3-1.7B layer, long context,
+ragged serving batch), the fused LM head, the end-to-end step through the public
+calls with host buffers, and the fp64 CPU oracle on a bounded sample.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -21,7 +31,6 @@ import ctypes
 import hashlib
 import json
 import os
-import re
 import statistics
 import subprocess
 import sys
@@ -42,7 +51,9 @@ UNIT = "GB/s"
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 ATTN_SRC = os.path.join(ROOT, "diffusion_draft_ar_b200", "csrc", "block_attn.cuh")
-TRAFFIC_SUMMARY = os.path.join(ROOT, "profiles", "block_attn_qwen3_8b.md")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "block_attn_qwen3_8b.json")
+NOMINAL_HBM_GBS = 8000.0        # the roofline the method's target is stated against
+NOMINAL_BF16_TFLOPS = 2250.0    # dense bf16 tensor peak (nominal)
 
 
 # ---------------------------------------------------------------------------
@@ -147,18 +158,64 @@ def measure_lm_head(O, w: W.Workload, m: W.BatchMeta, dev, stream, calls: int = 
 
 
 def traffic_per_launch():
-    """DRAM bytes per attention launch from the committed ncu summary, or None if
-    the summary is missing or was taken on a different kernel source."""
+    """DRAM bytes per attention launch from the committed ncu figures
+    (profiles/block_attn_qwen3_8b.json), or None when they are missing or were
+    taken on a different kernel source."""
     try:
-        txt = open(TRAFFIC_SUMMARY).read()
+        with open(TRAFFIC_FILE) as f:
+            d = json.load(f)
         src_hash = hashlib.sha256(open(ATTN_SRC, "rb").read()).hexdigest()[:16]
-        m = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]+)", txt)
-        t = re.search(r"dram_bytes_per_launch_full_size:\s*([0-9]+)", txt)
-        if m and t and m.group(1) == src_hash:
-            return int(t.group(1))
+        if d.get("kernel_source_sha256_16") == src_hash:
+            return int(d["dram_bytes_per_launch_full_size"])
     except Exception:
         pass
     return None
+
+
+class L2Scrub:
+    """Leaves L2 cold and clean before a timed call: a 256 MB write evicts every
+    line, then a 256 MB read of another buffer makes the write-backs of those
+    dirty lines happen before the call, and L2 ends holding clean lines of an
+    unrelated buffer. (A write alone would leave ~126 MB of dirty lines whose
+    write-back lands inside the next call: on this pool it slows a bare TMA
+    stream over the Qwen3-8B cache from 84 to 100 us.)"""
+
+    def __init__(self, dev, mb: int = 256):
+        self.a = torch.empty(mb << 20, dtype=torch.uint8, device=dev)
+        self.b = torch.ones(mb << 18, dtype=torch.float32, device=dev)
+        self.sink = torch.zeros(1, dtype=torch.float32, device=dev)
+
+    def __call__(self):
+        self.a.fill_(1)
+        torch.sum(self.b, 0, keepdim=True, out=self.sink)
+
+
+def timed_calls(calls, n: int, scrub: L2Scrub, stream, before=None):
+    """Run `n` steps of `calls` (a list of zero-argument functions), scrubbing L2
+    before each call; CUDA events on `stream` bracket each call alone. Returns
+    an [n, len(calls)] array of milliseconds."""
+    evs = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in calls] for _ in range(n)]
+    for i in range(n):
+        if before is not None:
+            before()
+        for j, f in enumerate(calls):
+            scrub()
+            evs[i][j][0].record(stream)
+            f()
+            evs[i][j][1].record(stream)
+    torch.cuda.synchronize()
+    return np.array([[e0.elapsed_time(e1) for e0, e1 in row] for row in evs])
+
+
+def hbm_roofline(nbytes: float, flops: float, us: float) -> dict:
+    """Achieved bandwidth and both roofline fractions: against the measured copy
+    bandwidth, and against max(bytes / 8 TB/s, FLOPs / 2.25 PFLOP/s)."""
+    peak, src = peak_hbm()
+    gbs = nbytes / (us * 1e-6) / 1e9
+    t_nom = max(nbytes / (NOMINAL_HBM_GBS * 1e9), flops / (NOMINAL_BF16_TFLOPS * 1e12))
+    return {"us": us, "gbs": gbs, "frac": gbs / peak, "peak_gbs": peak, "peak_source": src,
+            "frac_8tbs": t_nom / (us * 1e-6)}
 
 
 class ClockSampler:
@@ -212,7 +269,7 @@ class OracleSample:
     """One sequence of the workload: both attention views, its consensus rows and
     its append, computed by the fp64 CPU oracle."""
 
-    def __init__(self, w: W.Workload, seed: int = 0):
+    def __init__(self, w: W.Workload, seed: int = 0, threads: int | None = None):
         import oracle
         self.oracle = oracle
         self.w1 = w.with_(B=1)
@@ -233,7 +290,7 @@ class OracleSample:
         for view in W.VIEW_NAMES:
             self.bytes += attn_bytes(self.w1, m)
         self.bytes += consensus_bytes(self.w1, m)
-        self.threads = oracle.default_threads()
+        self.threads = threads or oracle.default_threads()
 
     def run(self) -> int:
         o, m = self.oracle, self.wi.meta
@@ -247,8 +304,8 @@ class OracleSample:
         return self.bytes + append_bytes(self.w1, int(acc.sum()))
 
 
-def cpu_baseline(w: W.Workload, budget_s: float = 10.0) -> dict:
-    s = OracleSample(w)
+def _time_oracle(w: W.Workload, budget_s: float, threads: int | None = None):
+    s = OracleSample(w, threads=threads)
     done, nbytes, t0 = 0, 0, time.perf_counter()
     while True:
         nbytes += s.run()
@@ -256,10 +313,25 @@ def cpu_baseline(w: W.Workload, budget_s: float = 10.0) -> dict:
         el = time.perf_counter() - t0
         if el >= budget_s or done >= w.B:
             break
-    return {"value": nbytes / el / 1e9, "unit": UNIT, "cores": s.threads, "kind": "oracle",
-            "sample": f"{done} sequence(s) of {w.name} (both attention views over L={w.prefix_len}, "
-                      f"consensus over {w.max_block} rows x V={w.vocab}, append), fp64 C oracle, "
-                      f"{el:.1f} s"}
+    return s, done, nbytes, el
+
+
+def cpu_baseline(w: W.Workload, budget_s: float = 10.0, single_thread: bool = True) -> dict:
+    s, done, nbytes, el = _time_oracle(w, budget_s)
+    out = {"value": nbytes / el / 1e9, "unit": UNIT, "cores": s.threads, "kind": "oracle",
+           "sample": f"{done} sequence(s) of {w.name} (both attention views over L={w.prefix_len}, "
+                     f"consensus over {w.max_block} rows x V={w.vocab}, append), fp64 C oracle, "
+                     f"{el:.1f} s"}
+    if single_thread:
+        # the same oracle on one host thread, on the two small workloads
+        st = {}
+        for name in ("tiny", "qwen3_1p7b"):
+            s1, d1, b1, e1 = _time_oracle(W.WORKLOADS[name], min(budget_s, 5.0), threads=1)
+            st[name] = {"value": b1 / e1 / 1e9, "unit": UNIT, "cores": 1,
+                        "ms_per_sequence": 1e3 * e1 / d1,
+                        "sample": f"{d1} sequence(s): both views, consensus, append"}
+        out["single_thread"] = st
+    return out
 
 
 def run_reference(args):
@@ -296,89 +368,174 @@ def run_reference(args):
 # ---------------------------------------------------------------------------
 # GPU arm
 
+class AttnCall:
+    """One prepared orthrus_block_attn (or _verify_write) call on device inputs."""
+
+    def __init__(self, O, view, q, k_cache, v_cache, kb, vb, lens, cu, table, max_block,
+                 err, stream, kv_split: int = 0, write: bool = False):
+        self.O = O
+        self.out = torch.empty_like(q)
+        self.p = O.attn_params(view, q, k_cache, v_cache, kb, vb, lens, cu, table, self.out,
+                               max_block, kv_split_tokens=kv_split, error_flag=err)
+        self.ws = torch.empty(max(256, O.block_attn_workspace_size(self.p)), dtype=torch.uint8,
+                              device=q.device)
+        self.p.workspace, self.p.workspace_bytes = self.ws.data_ptr(), self.ws.numel()
+        self.kernels = O.block_attn_kernel_count(self.p)
+        self.P = ctypes.byref(self.p)
+        self.sp = ctypes.c_void_p(stream.cuda_stream)
+        self.fn = O.lib.orthrus_block_attn_verify_write if write else O.lib.orthrus_block_attn
+
+    def __call__(self):
+        st = self.fn(self.P, self.sp)
+        if st:
+            raise RuntimeError(f"attention call failed: {self.O.lib.orthrus_last_error().decode()}")
+
+
+class ConsensusCall:
+    def __init__(self, O, logits, drafts, cu, B, max_block, stream, lens=None):
+        dev = logits.device
+        self.O = O
+        self.acc = torch.zeros(B, dtype=torch.int32, device=dev)
+        self.nxt = torch.zeros(B, dtype=torch.int32, device=dev)
+        self.ws = torch.empty(O.consensus_workspace_size(B, max_block, logits.shape[1]),
+                              dtype=torch.uint8, device=dev)
+        sp = ctypes.c_void_p(stream.cuda_stream)
+        V = logits.shape[1]
+        base = (logits.data_ptr(), V, V, drafts.data_ptr(), cu.data_ptr(), B, max_block,
+                self.acc.data_ptr(), self.nxt.data_ptr(), None)
+        if lens is None:
+            self.fn, self.args = O.lib.orthrus_consensus, base + (self.ws.data_ptr(),
+                                                                  self.ws.numel(), sp)
+        else:
+            self.fn, self.args = O.lib.orthrus_consensus_commit, base + (
+                lens.data_ptr(), self.ws.data_ptr(), self.ws.numel(), sp)
+
+    def __call__(self):
+        st = self.fn(*self.args)
+        if st:
+            raise RuntimeError(f"consensus failed: {self.O.lib.orthrus_last_error().decode()}")
+
+
+def check_flag(err, what):
+    v = int(err.item())
+    if v:
+        raise RuntimeError(f"{what}: device error flag {v}")
+
+
+def measure_workload(O, name: str, dev, stream, scrub, calls: int, seed: int = 0) -> dict:
+    """Per-call times (L2 scrubbed before each call) of one workload's attention
+    views, and, where the workload has a vocabulary, its consensus and a whole
+    round (DIFFUSION, write-then-truncate VERIFY, consensus with commit)."""
+    w = W.WORKLOADS[name]
+    wi = W.WorkloadInputs(w, device=dev, seed=seed, rounds=1)
+    m, r = wi.meta, wi.rounds[0]
+    lens0 = m.prefix_lens.to(dev)
+    lens = lens0.clone()
+    cu, table = m.cu_block.to(dev), m.page_table.to(dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    kv = int(m.prefix_lens.to(torch.int64).sum()) * W.cache_bytes_per_token(w)
+    res = {"workload": name, "B": m.B, "rows": m.R, "prefix_tokens": int(m.prefix_lens.sum()),
+           "kv_bytes": kv, "calls": calls, "views": {}}
+    b_attn = attn_bytes(w, m)
+    for view in w.views:
+        variants = [("library schedule", 0)]
+        if w.kv_split_tokens:
+            variants.append((f"{w.kv_split_tokens}-token chunks", w.kv_split_tokens))
+        for label, split in variants:
+            c = AttnCall(O, view, r.q[view], wi.k_cache, wi.v_cache, r.k_block[view],
+                         r.v_block[view], lens, cu, table, w.max_block, err, stream,
+                         kv_split=split)
+            for _ in range(3):
+                scrub(); c()
+            t = timed_calls([c], calls, scrub, stream)[:, 0]
+            check_flag(err, f"{name}/{view}")
+            us = float(np.median(t)) * 1e3
+            d = hbm_roofline(b_attn, attn_flops(w, m, view), us)
+            d.update({"us_mean": float(t.mean()) * 1e3, "kernels": c.kernels,
+                      "algorithmic_bytes": b_attn, "blocks_per_s": m.B / (us * 1e-6),
+                      "tokens_verified_per_s": m.R / (us * 1e-6) if view == "verify" else None})
+            res["views"][view if len(variants) == 1 else f"{view} ({label})"] = d
+    if w.vocab is not None and set(w.views) == set(W.VIEW_NAMES):
+        targets = torch.argmax(r.logits, dim=1).to(torch.int32)
+        drafts = wi.drafts(0, targets)
+        diff = AttnCall(O, "diffusion", r.q["diffusion"], wi.k_cache, wi.v_cache,
+                        r.k_block["diffusion"], r.v_block["diffusion"], lens, cu, table,
+                        w.max_block, err, stream)
+        ver = AttnCall(O, "verify", r.q["verify"], wi.k_cache, wi.v_cache, r.k_block["verify"],
+                       r.v_block["verify"], lens, cu, table, w.max_block, err, stream,
+                       write=True)
+        cons = ConsensusCall(O, r.logits, drafts, cu, m.B, w.max_block, stream, lens=lens)
+        restore = lambda: lens.copy_(lens0, non_blocking=True)
+        for _ in range(3):
+            restore()
+            for f in (diff, ver, cons):
+                scrub(); f()
+        t = timed_calls([diff, ver, cons], calls, scrub, stream, before=restore)
+        check_flag(err, f"{name} round")
+        t_c = float(np.median(t[:, 2])) * 1e3
+        b_c = consensus_bytes(w, m)
+        round_us = float(np.median(t.sum(1))) * 1e3
+        res["consensus"] = {"us": t_c, "gbs": b_c / (t_c * 1e-6) / 1e9,
+                            "frac": b_c / (t_c * 1e-6) / 1e9 / peak_hbm()[0],
+                            "rows_per_s": m.R / (t_c * 1e-6), "algorithmic_bytes": b_c}
+        res["round"] = {"us": round_us, "blocks_per_s": m.B / (round_us * 1e-6),
+                        "tokens_verified_per_s": m.R / (round_us * 1e-6),
+                        "mean_accept_len": float(cons.acc.float().mean()),
+                        "calls": "DIFFUSION attention, write-then-truncate VERIFY attention, "
+                                 "consensus with commit"}
+    del wi
+    torch.cuda.empty_cache()
+    return res
+
+
 def run_ours(args):
     world, rank, local = D.init("nccl", timeout_s=300)
     from diffusion_draft_ar_b200 import orthrus as O
     w = W.WORKLOADS[args.workload]
     dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream()
+    scrub = L2Scrub(dev)
     wi = W.WorkloadInputs(w, device=dev, seed=D.rank_seed(0, rank))
     m, r = wi.meta, wi.rounds[0]
-    stream = torch.cuda.current_stream()
     lens0 = m.prefix_lens.to(dev)
     lens = lens0.clone()
     cu = m.cu_block.to(dev)
     table = m.page_table.to(dev)
     err = torch.zeros(1, dtype=torch.int32, device=dev)
-    outs, params = {}, {}
-    ws_attn = None
-    for view in W.VIEW_NAMES:
-        outs[view] = torch.empty_like(r.q[view])
-        p = O.attn_params(view, r.q[view], wi.k_cache, wi.v_cache, r.k_block[view],
-                          r.v_block[view], lens, cu, table, outs[view], w.max_block,
-                          kv_split_tokens=w.kv_split_tokens, error_flag=err)
-        n = O.block_attn_workspace_size(p)
-        if ws_attn is None or ws_attn.numel() < n:
-            ws_attn = torch.empty(n, dtype=torch.uint8, device=dev)
-        params[view] = p
-    for p in params.values():
-        p.workspace, p.workspace_bytes = ws_attn.data_ptr(), ws_attn.numel()
-    # our kernels per step: both attention calls (1 or 2 kernels each),
-    # consensus (argmax + finalize) and, when the commit is a separate append, kv_append
     write = args.commit == "write"
-    launches_per_step = (sum(O.block_attn_kernel_count(p) for p in params.values()) + 2 +
-                         (0 if write else 1))
     targets = torch.argmax(r.logits, dim=1).to(torch.int32)
     drafts = wi.drafts(0, targets)
-    acc = torch.zeros(m.B, dtype=torch.int32, device=dev)
-    nxt = torch.zeros(m.B, dtype=torch.int32, device=dev)
-    ws_cons = torch.empty(O.consensus_workspace_size(m.B, w.max_block, w.vocab),
-                          dtype=torch.uint8, device=dev)
-    L = O.lib
+    diff = AttnCall(O, "diffusion", r.q["diffusion"], wi.k_cache, wi.v_cache,
+                    r.k_block["diffusion"], r.v_block["diffusion"], lens, cu, table, w.max_block,
+                    err, stream, kv_split=w.kv_split_tokens)
+    ver = AttnCall(O, "verify", r.q["verify"], wi.k_cache, wi.v_cache, r.k_block["verify"],
+                   r.v_block["verify"], lens, cu, table, w.max_block, err, stream,
+                   kv_split=w.kv_split_tokens, write=write)
+    cons = ConsensusCall(O, r.logits, drafts, cu, m.B, w.max_block, stream,
+                         lens=lens if write else None)
     sp = ctypes.c_void_p(stream.cuda_stream)
-    P_diff, P_ver = ctypes.byref(params["diffusion"]), ctypes.byref(params["verify"])
-    cons_args = (r.logits.data_ptr(), w.vocab, w.vocab, drafts.data_ptr(), cu.data_ptr(), m.B,
-                 w.max_block, acc.data_ptr(), nxt.data_ptr(), None, ws_cons.data_ptr(),
-                 ws_cons.numel(), sp)
-    commit_args = cons_args[:10] + (lens.data_ptr(),) + cons_args[10:]
     kb, vb = r.k_block["verify"], r.v_block["verify"]
-    app_args = (kb.data_ptr(), vb.data_ptr(), cu.data_ptr(), w.max_block, acc.data_ptr(),
+    app_args = (kb.data_ptr(), vb.data_ptr(), cu.data_ptr(), w.max_block, cons.acc.data_ptr(),
                 lens.data_ptr(), 1, table.data_ptr(), m.max_pages, m.num_pages,
                 wi.k_cache.data_ptr(), wi.v_cache.data_ptr(), m.B, w.Hkv, w.D, w.page_size,
                 err.data_ptr(), sp)
 
-    def step(ev=None):
-        lens.copy_(lens0, non_blocking=True)
-        if ev is not None:
-            ev[0].record(stream)
-        s1 = L.orthrus_block_attn(P_diff, sp)
-        if ev is not None:
-            ev[1].record(stream)
-        if write:  # write-then-truncate: VERIFY stores the block K/V, consensus commits
-            s2 = L.orthrus_block_attn_verify_write(P_ver, sp)
-        else:
-            s2 = L.orthrus_block_attn(P_ver, sp)
-        if ev is not None:
-            ev[2].record(stream)
-        if write:
-            s3 = L.orthrus_consensus_commit(*commit_args)
-        else:
-            s3 = L.orthrus_consensus(*cons_args)
-        if ev is not None:
-            ev[3].record(stream)
-        s4 = 0 if write else L.orthrus_kv_append(*app_args)
-        if ev is not None:
-            ev[4].record(stream)
-        if s1 or s2 or s3 or s4:
-            raise RuntimeError(f"orthrus call failed: {(s1, s2, s3, s4)} "
-                               f"{L.orthrus_last_error().decode()}")
+    def append():
+        st = O.lib.orthrus_kv_append(*app_args)
+        if st:
+            raise RuntimeError(f"kv_append failed: {O.lib.orthrus_last_error().decode()}")
+
+    step_calls = [diff, ver, cons] + ([] if write else [append])
+    launches_per_step = diff.kernels + ver.kernels + 2 + (0 if write else 1)
+    restore = lambda: lens.copy_(lens0, non_blocking=True)
 
     for _ in range(args.warmup):
-        step()
+        restore()
+        for f in step_calls:
+            scrub(); f()
     torch.cuda.synchronize()
-    if int(err.item()) != 0:
-        raise RuntimeError(f"device error flag {int(err.item())}")
+    check_flag(err, "warm-up")
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(dev.index)
@@ -387,27 +544,39 @@ def run_ours(args):
     D.barrier(world)
     torch.cuda.synchronize()
     t_start.record(stream)
-    for i in range(args.steps):
-        step(evs[i])
+    part = timed_calls(step_calls, args.steps, scrub, stream, before=restore)  # ms
     t_end.record(stream)
     torch.cuda.synchronize()
     D.barrier(world)
     clocks = sampler.stop()
-    total_ms = t_start.elapsed_time(t_end)
-    part = np.array([[e[j].elapsed_time(e[j + 1]) for j in range(4)] for e in evs])  # ms
-    total_ms = D.max_over_ranks(total_ms, world)
-    ms_step = total_ms / args.steps
-    t_diff, t_ver, t_cons, t_app = (float(x) for x in part.mean(0))
+    check_flag(err, "timed steps")
+    wall_ms = D.max_over_ranks(t_start.elapsed_time(t_end), world) / args.steps
+    ms_step = D.max_over_ranks(float(part.sum(1).mean()), world)
+    t_diff, t_ver, t_cons = (float(x) for x in part[:, :3].mean(0))
+    t_app = float(part[:, 3].mean()) if not write else None
 
-    accepted = int(acc.sum().item())
+    accepted = int(cons.acc.sum().item())
     mean_accept = accepted / m.B
     b_attn = attn_bytes(w, m)
     b_step = 2 * b_attn + consensus_bytes(w, m) + append_bytes(w, accepted)
     value = world * b_step / (ms_step * 1e-3) / 1e9
     attn_ms = 0.5 * (t_diff + t_ver)
-    attn_gbs = b_attn / (attn_ms * 1e-3) / 1e9
-    peak, peak_src = peak_hbm()
     flops = 0.5 * (attn_flops(w, m, "diffusion") + attn_flops(w, m, "verify"))
+    roof_att = hbm_roofline(b_attn, flops, attn_ms * 1e3)
+
+    # ---- the separate append launch on the same rows (accept lengths of the last step)
+    app_calls = 50
+    for _ in range(3):
+        restore(); scrub(); append()
+    t = timed_calls([append], app_calls, scrub, stream, before=restore)[:, 0]
+    check_flag(err, "kv_append")
+    app_us = float(np.median(t)) * 1e3
+    b_app = append_bytes(w, accepted)
+    kv_append = {"us": app_us, "gbs": b_app / (app_us * 1e-6) / 1e9,
+                 "frac": b_app / (app_us * 1e-6) / 1e9 / peak_hbm()[0],
+                 "algorithmic_bytes": b_app, "accepted_rows": accepted, "calls": app_calls,
+                 "note": "orthrus_kv_append of the accepted VERIFY rows (K and V, read + write), "
+                         "prefix lengths restored before each call; latency-bound at this size"}
 
     # ---- end to end through the public API: pinned host inputs in, results out ----
     e2e_steps = max(1, min(args.steps, args.e2e_steps))
@@ -418,11 +587,11 @@ def run_ours(args):
     d_in = {"qd": r.q["diffusion"], "kd": r.k_block["diffusion"], "vd": r.v_block["diffusion"],
             "qv": r.q["verify"], "kv": r.k_block["verify"], "vv": r.v_block["verify"],
             "logits": r.logits, "drafts": drafts}
-    h_out = {"od": torch.empty_like(outs["diffusion"], device="cpu").pin_memory(),
-             "ov": torch.empty_like(outs["verify"], device="cpu").pin_memory(),
-             "acc": torch.empty_like(acc, device="cpu").pin_memory(),
-             "nxt": torch.empty_like(nxt, device="cpu").pin_memory()}
-    d_out = {"od": outs["diffusion"], "ov": outs["verify"], "acc": acc, "nxt": nxt}
+    h_out = {"od": torch.empty_like(diff.out, device="cpu").pin_memory(),
+             "ov": torch.empty_like(ver.out, device="cpu").pin_memory(),
+             "acc": torch.empty_like(cons.acc, device="cpu").pin_memory(),
+             "nxt": torch.empty_like(cons.nxt, device="cpu").pin_memory()}
+    d_out = {"od": diff.out, "ov": ver.out, "acc": cons.acc, "nxt": cons.nxt}
     h2d = sum(t.numel() * t.element_size() for t in h_in.values())
     d2h = sum(t.numel() * t.element_size() for t in h_out.values())
     e0 = torch.cuda.Event(enable_timing=True)
@@ -433,14 +602,25 @@ def run_ours(args):
     for _ in range(e2e_steps):
         for k in h_in:
             d_in[k].copy_(h_in[k], non_blocking=True)
-        step()
+        restore()
+        for f in step_calls:
+            f()
         for k in h_out:
             h_out[k].copy_(d_out[k], non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
     D.barrier(world)
+    check_flag(err, "e2e")
     e2e_ms = D.max_over_ranks(e0.elapsed_time(e1), world) / e2e_steps
     e2e_value = world * b_step / (e2e_ms * 1e-3) / 1e9
+    del wi, h_in, h_out
+    torch.cuda.empty_cache()
+
+    # ---- the other workloads, each timed alone ----
+    configs = {}
+    if not args.no_configs:
+        for name in ("qwen3_1p7b", "longctx", "ragged"):
+            configs[name] = measure_workload(O, name, dev, stream, scrub, args.config_calls)
 
     lm_head = None if args.no_lm_head else measure_lm_head(O, w, m, dev, stream)
 
@@ -448,20 +628,15 @@ def run_ours(args):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, budget_s=args.cpu_seconds)
 
-    cache_mb = 2 * wi.k_cache.numel() * wi.k_cache.element_size() / 1e6
-    logits_mb = r.logits.numel() * r.logits.element_size() / 1e6
-    if cache_mb + logits_mb > 126.0:
-        l2_note = (f"inputs larger than L2 (KV cache {cache_mb:.0f} MB, logits "
-                   f"{logits_mb:.0f} MB), no flush")
-    else:
-        l2_note = (f"inputs fit in L2 (KV cache {cache_mb:.0f} MB, logits {logits_mb:.0f} MB): "
-                   f"back-to-back timing, L2-resident")
     if rank == 0:
-        roof = {"bound": "hbm", "achieved": attn_gbs, "peak": peak, "unit": "GB/s",
-                "frac": attn_gbs / peak, "traffic": traffic_per_launch(),
+        roof = {"bound": "hbm", "achieved": roof_att["gbs"], "peak": roof_att["peak_gbs"],
+                "unit": "GB/s", "frac": roof_att["frac"], "frac_8tbs": roof_att["frac_8tbs"],
+                "traffic": traffic_per_launch(),
                 "kernel": "orthrus_block_attn (attention + split combine), mean of both views",
                 "algorithmic_bytes_per_launch": b_attn, "us_per_launch": attn_ms * 1e3,
-                "peak_source": f"{peak_src} HBM copy bandwidth",
+                "peak_source": f"{roof_att['peak_source']} HBM copy bandwidth (MEASURED_PEAKS)",
+                "frac_8tbs_definition": "max(bytes / 8 TB/s, FLOPs / 2.25 PFLOP/s) / time",
+                "l2": "scrubbed before every launch",
                 "tensor_tflops": flops / (attn_ms * 1e-3) / 1e12}
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -473,12 +648,17 @@ def run_ours(args):
                        "vocab": w.vocab,
                        "pages": "random permutation" if w.paged else "contiguous",
                        "parallelism": f"dp{world} (independent batches)",
-                       "l2": l2_note},
-            "block_attn_gbs": attn_gbs, "block_attn_us": {"diffusion": t_diff * 1e3,
-                                                          "verify": t_ver * 1e3},
+                       "l2": "flushed before every timed call (256 MB write, then 256 MB read "
+                             "of another buffer, outside the timed interval); ms_per_step is "
+                             "the sum of the calls' event-timed intervals"},
+            "ms_per_step_incl_flush": wall_ms,
+            "block_attn_gbs": roof_att["gbs"], "block_attn_us": {"diffusion": t_diff * 1e3,
+                                                                 "verify": t_ver * 1e3},
             "consensus_rows_per_s": world * m.R / (t_cons * 1e-3),
             "consensus_us": t_cons * 1e3,
-            "kv_append_us": None if write else t_app * 1e3,
+            "consensus_gbs": consensus_bytes(w, m) / (t_cons * 1e-3) / 1e9,
+            "kv_append_us": t_app * 1e3 if t_app is not None else None,
+            "kv_append": kv_append,
             "commit": ("write-then-truncate (VERIFY attention stores the block K/V; "
                        "consensus advances the lengths)") if write else
                       "separate kv_append of the accepted rows",
@@ -486,12 +666,13 @@ def run_ours(args):
             "tokens_verified_per_s": world * m.R / (t_ver * 1e-3),
             "mean_accept_len": mean_accept,
             "roofline": roof,
+            "configs": configs,
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": e2e_steps, "ms_per_step": e2e_ms,
                     "note": "per step: pinned H2D of both views' q/k/v blocks, logits and drafts; "
                             "D2H of both outputs, accept lengths and next tokens; "
-                            "the KV cache stays resident"},
+                            "the KV cache stays resident; no L2 flush"},
             "gpu_launches": args.steps * launches_per_step,
             "lm_head": lm_head,
             "clocks": clocks,
@@ -503,7 +684,7 @@ def run_ours(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     # the step needs both attention views and a vocabulary (longctx is VERIFY-only
@@ -516,6 +697,10 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-lm-head", action="store_true",
                     help="skip the separate fused LM-head measurement")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the Qwen3-1.7B, long-context and ragged measurements")
+    ap.add_argument("--config-calls", type=int, default=20,
+                    help="timed calls per measurement on the other workloads")
     ap.add_argument("--commit", choices=["write", "append"], default="write",
                     help="write: VERIFY attention stores the block K/V and consensus advances "
                          "the lengths (write-then-truncate); append: separate kv_append launch")

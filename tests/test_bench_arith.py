@@ -54,19 +54,35 @@ def test_consensus_and_append_bytes(q8):
     assert bench.append_bytes(w, 1) == 2 * 2 * w.Hkv * w.D * 2 == 8192
 
 
-def test_traffic_parser_follows_the_kernel_hash(monkeypatch):
-    """The bench reports DRAM traffic only while the committed ncu summary was
+def test_traffic_file_follows_the_kernel_hash(monkeypatch):
+    """The bench reports DRAM traffic only while the committed ncu figures were
     taken on the current kernel source."""
-    src = b"// kernel source\n"
     import hashlib
+    import json
+    src = b"// kernel source\n"
     h = hashlib.sha256(src).hexdigest()[:16]
     with tempfile.TemporaryDirectory() as d:
         k = os.path.join(d, "k.cuh")
         open(k, "wb").write(src)
-        s = os.path.join(d, "s.md")
-        open(s, "w").write(f"kernel_source_sha256_16: {h}\ndram_bytes_per_launch_full_size: 1234\n")
+        s = os.path.join(d, "s.json")
+        json.dump({"kernel_source_sha256_16": h, "dram_bytes_per_launch_full_size": 1234},
+                  open(s, "w"))
         monkeypatch.setattr(bench, "ATTN_SRC", k)
-        monkeypatch.setattr(bench, "TRAFFIC_SUMMARY", s)
+        monkeypatch.setattr(bench, "TRAFFIC_FILE", s)
         assert bench.traffic_per_launch() == 1234
         open(k, "wb").write(src + b"// changed\n")
         assert bench.traffic_per_launch() is None
+
+
+def test_roofline_fractions():
+    """Both fractions from their definitions: against the measured copy
+    bandwidth, and against max(bytes / 8 TB/s, FLOPs / 2.25 PFLOP/s)."""
+    nbytes, flops, us = 547_356_672, 68_987_912_192, 100.0
+    d = bench.hbm_roofline(nbytes, flops, us)
+    assert abs(d["gbs"] - 5473.56672) < 1e-6
+    assert abs(d["frac"] - d["gbs"] / bench.peak_hbm()[0]) < 1e-12
+    # bytes / 8 TB/s = 68.42 us dominates FLOPs / 2.25 PF = 30.66 us
+    assert abs(d["frac_8tbs"] - (nbytes / 8e12) / 100e-6) < 1e-12
+    # a compute-heavy case takes the FLOP term
+    d2 = bench.hbm_roofline(1e6, 2.25e9, 10.0)
+    assert abs(d2["frac_8tbs"] - (2.25e9 / 2.25e15) / 10e-6) < 1e-12
