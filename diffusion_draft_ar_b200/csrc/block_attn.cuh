@@ -584,34 +584,14 @@ __device__ __forceinline__ void producer_role(const AttnArgs& a, uint8_t* smem,
   }
 }
 
-// One step of the MMA issuer's walk over the CTA's tiles.
+// One tile as the MMA issuer sees it: its unit segment, its index inside the
+// unit (t) and in the CTA's tile order (it), and the unit's lengths.
 struct TileStep {
   SegCursor cur;
   Segment sg;
   int si, t, it, L, np, Kb;
   bool valid;
 };
-
-__device__ __forceinline__ bool step_next(const AttnArgs& a, const SeqTable& tab, TileStep& s) {
-  if (s.valid && s.t + 1 < s.sg.t1) {
-    ++s.t;
-    ++s.it;
-    return true;
-  }
-  if (!cursor_next(a, tab, s.cur, s.sg)) {
-    s.valid = false;
-    return false;
-  }
-  ++s.si;
-  ++s.it;
-  s.t = s.sg.t0;
-  const SeqInfo sq = tab.get(a, s.sg.b);
-  s.L = sq.L;
-  s.np = (s.L + kTileN - 1) / kTileN;
-  s.Kb = sq.Kb;
-  s.valid = true;
-  return true;
-}
 
 // One MMA warp per softmax group w: it issues QK and PV for the group's tiles
 // (global tile index parity w). The issuing thread's scalar work sits between
@@ -622,8 +602,6 @@ __device__ __forceinline__ bool step_next(const AttnArgs& a, const SeqTable& tab
 // Q bookkeeping covers every segment, own tiles or not: at a segment start the
 // warp waits for that unit's Q tile, and after its last QK of the segment it
 // commits one arrival on q_empty (two arrivals, one per warp, release Q).
-// Waiting for the next Q before committing for it keeps one warp from
-// completing a q_empty phase on its own.
 template <int D>
 __device__ __forceinline__ void mma_role(const AttnArgs& a, uint8_t* smem, uint32_t tmem,
                                          volatile int* abort_flag, int w, const SeqTable& tab,
@@ -709,62 +687,65 @@ __device__ __forceinline__ void mma_role(const AttnArgs& a, uint8_t* smem, uint3
     return true;
   };
 
-  // QK walk over every tile: Q waits and commits at segment edges, QK for own
-  // tiles, up to two own tiles ahead of PV. The walk holds at the end of a
-  // unit while PVs of that unit are still to be issued: they go first, so the
-  // unit's last PVs (and the epilogue waiting on them) never queue behind the
-  // next unit's QKs, which must wait for that unit's Q tile to load.
-  TileStep qs;
-  qs.cur = start;
-  qs.si = -1;
-  qs.it = -1;
-  qs.valid = false;
-  TileStep ps = qs;
-  int mq = 0, mp = 0;  // own tiles issued (QK) / (PV)
-  bool ok = true, qk_pending = false, qk_done = false;
+  // The CTA's range is walked one unit segment at a time, and within a
+  // segment this warp's own tiles (CTA tile index it = w, w + 2, ...) in a
+  // straight loop: QK(0), QK(1), then PV(m), QK(m + 2) for m = 0, 1, ... (the
+  // QKs run two own tiles ahead of the PVs, the depth of the S double buffer).
+  // A segment's QKs start only after every PV of the previous segment was
+  // issued, so the unit's last PVs (and the epilogue waiting on them) never
+  // queue behind the next unit's QKs, which wait for that unit's Q tile.
+  // The per-tile bookkeeping is a few integer operations: this warp's issue
+  // loop paces the whole pipeline (a general tile walker here, with its
+  // branches between the MMA batches, cost about 12% of a Qwen3-8B layer).
   auto commit_q_empty = [&]() {
     if (elect_one()) mma_commit(bars + 8u * Lay::kBarQEmpty);
     __syncwarp();
   };
-  auto walk_qk = [&]() {  // move qs to the next own tile
-    while (ok) {
-      if (qs.valid && qs.t + 1 >= qs.sg.t1 && mp < mq) return;  // hold at the unit's end
-      if (!step_next(a, tab, qs)) {
-        qk_done = true;
-        return;
+  SegCursor cur = start;
+  Segment sg;
+  int si = 0;   // segment index (Q tile and O phases)
+  int it0 = 0;  // CTA tile index of the segment's first tile
+  int mb = 0;   // own tiles of this warp in earlier segments
+  bool ok = true;
+  while (ok && cursor_next(a, tab, cur, sg)) {
+    const SeqInfo sq = tab.get(a, sg.b);
+    TileStep j;
+    j.cur = cur;
+    j.sg = sg;
+    j.si = si;
+    j.L = sq.L;
+    j.np = (sq.L + kTileN - 1) / kTileN;
+    j.Kb = sq.Kb;
+    j.valid = true;
+    const int n = sg.t1 - sg.t0;
+    const int first = (w - it0) & 1;  // segment-local index of the first own tile
+    const int n_own = n > first ? (n - first + 1) / 2 : 0;
+    auto tile = [&](int m) {  // own tile m of the segment
+      TileStep x = j;
+      const int loc = first + 2 * m;
+      x.t = sg.t0 + loc;
+      x.it = it0 + loc;
+      return x;
+    };
+    // Every warp waits for the unit's Q tile, own tiles or not, before it
+    // commits its release: one warp never completes a q_empty phase alone.
+    if (!wait(bars + 8u * Lay::kBarQFull, si & 1)) { ok = false; break; }
+    for (int m = 0; m < 2 && m < n_own && ok; ++m) ok = issue_qk(tile(m), mb + m);
+    if (!ok) break;
+    if (n_own <= 2) commit_q_empty();
+    for (int m = 0; m < n_own && ok; ++m) {
+      // the group's first PV of a unit overwrites O: the previous unit's
+      // epilogue must have read it
+      if (m == 0 && si > 0 && !wait(bars + 8u * Lay::kBarOFree, (si - 1) & 1)) { ok = false; break; }
+      ok = issue_pv(tile(m), mb + m);
+      if (ok && m + 2 < n_own) {
+        ok = issue_qk(tile(m + 2), mb + m + 2);
+        if (ok && m + 3 == n_own) commit_q_empty();
       }
-      if (qs.t == qs.sg.t0 && !wait(bars + 8u * Lay::kBarQFull, qs.si & 1)) { ok = false; return; }
-      if ((qs.it & 1) == w) {
-        qk_pending = true;
-        return;
-      }
-      if (qs.t == qs.sg.t1 - 1) commit_q_empty();
     }
-  };
-  auto try_qk = [&]() -> bool {  // issue the next own QK unless held
-    if (!qk_pending && !qk_done) walk_qk();
-    if (!ok || !qk_pending) return false;
-    if (!issue_qk(qs, mq)) { ok = false; return false; }
-    ++mq;
-    qk_pending = false;
-    if (qs.t == qs.sg.t1 - 1) commit_q_empty();
-    return true;
-  };
-  auto advance_pv = [&]() -> bool {
-    while (ok && step_next(a, tab, ps)) {
-      if ((ps.it & 1) != w) continue;
-      if (ps.t <= ps.sg.t0 + 1 && ps.si > 0 &&
-          !wait(bars + 8u * Lay::kBarOFree, (ps.si - 1) & 1)) { ok = false; break; }
-      if (!issue_pv(ps, mp)) { ok = false; break; }
-      ++mp;
-      return true;
-    }
-    return false;
-  };
-  while (ok) {
-    while (ok && mq - mp < 2 && try_qk()) {}
-    if (!ok || mp == mq) break;  // every QK issued (walk done) and every PV too
-    if (!advance_pv()) break;
+    mb += n_own;
+    it0 += n;
+    ++si;
   }
   // Drain: every MMA issued above completes before TMEM is released.
   if (elect_one()) {
@@ -844,9 +825,9 @@ __device__ __forceinline__ void softmax_role(const AttnArgs& a, uint8_t* smem, u
 #pragma unroll
       for (int k = 0; k < 8; ++k) mx[k] = s[k];
 #pragma unroll
-      for (int k = 8; k < 64; ++k) mx[k & 7] = fmaxf(mx[k & 7], s[k]);
-      const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                             fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+      for (int k = 8; k < 64; k += 2) mx[(k >> 1) & 7] = fmax3(mx[(k >> 1) & 7], s[k], s[k + 1]);
+      const float mt = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]),
+                             fmaxf(mx[6], mx[7]));
       const float m_new = fmaxf(m_ref, mt * c);
       const bool need = has && (m_new > m_ref + kRescaleLog2);
       if (!has) m_ref = m_new;
@@ -889,18 +870,25 @@ __device__ __forceinline__ void softmax_role(const AttnArgs& a, uint8_t* smem, u
         tmem_wait_st();
       }
       const float mref = (m_ref == NEG_INF) ? 0.f : m_ref;
-      float psum[8];
+      // Scale-and-subtract and the row sums run as packed fp32 pairs and the
+      // maximum as three-input max, which cuts the softmax warps' instruction
+      // count per tile by about a third; the arithmetic (fp32 round-to-nearest
+      // FMA, the same eight partial sums in the same order) is unchanged.
+      float2 ps2[4];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) psum[k] = 0.f;
+      for (int k = 0; k < 4; ++k) ps2[k] = make_float2(0.f, 0.f);
       uint32_t pk[32];
+      const float2 c2 = make_float2(c, c), nm2 = make_float2(-mref, -mref);
 #pragma unroll
       for (int k = 0; k < 32; ++k) {
-        const float p0 = ex2_approx(fmaf(s[2 * k], c, -mref));
-        const float p1 = ex2_approx(fmaf(s[2 * k + 1], c, -mref));
-        psum[(2 * k) & 7] += p0;
-        psum[(2 * k + 1) & 7] += p1;
-        pk[k] = pack_bf16x2(p0, p1);
+        const float2 x = ffma2(make_float2(s[2 * k], s[2 * k + 1]), c2, nm2);
+        const float2 p = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+        ps2[k & 3] = fadd2(ps2[k & 3], p);
+        pk[k] = pack_bf16x2(p.x, p.y);
       }
+      float psum[8];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) psum[2 * k] = ps2[k].x, psum[2 * k + 1] = ps2[k].y;
       // P (bf16 pairs) over the first 32 columns of this tile's S buffer
       tmem_st32u(t_s, pk);
       if (!wait(bars + 8u * (Lay::kBarVFull + it % Lay::kNV), (it / Lay::kNV) & 1)) {
