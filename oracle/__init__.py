@@ -28,6 +28,11 @@ Dual-View Diffusion, technical summary):
   vocabulary, and its greedy token is the first index of the largest score.
 * ``accept_from_tokens`` -- the §2.3 item 3 rule of ``consensus`` applied to
   given greedy tokens.
+* ``consensus_sampled`` / ``sampled_tokens`` -- temperature > 0 (the pages
+  name temperature settings, §4, but give no sampling rule; the reading
+  taken): the AR token of each row is a Gumbel-max sample from
+  softmax(logits / T), with uniforms from Philox4x32-10 (``philox4x32_10``,
+  Salmon et al., SC 2011), and the §2.3 item 3 acceptance runs on it.
 """
 from __future__ import annotations
 
@@ -89,6 +94,14 @@ def _load():
         lib.oracle_lm_head.argtypes = [p, p, i32, i32, p, i64, p, p, i32]
         lib.oracle_greedy_tokens.restype = None
         lib.oracle_greedy_tokens.argtypes = [p, i64, i32, p]
+        u64 = ctypes.c_uint64
+        lib.oracle_philox4x32_10.restype = None
+        lib.oracle_philox4x32_10.argtypes = [p, p, p]
+        lib.oracle_sampled_tokens.restype = i32
+        lib.oracle_sampled_tokens.argtypes = [p, i64, i32, i64, dbl, u64, u64, p, p, i32]
+        lib.oracle_consensus_sampled.restype = i32
+        lib.oracle_consensus_sampled.argtypes = [p, i64, i32, p, p, i32, dbl, u64, u64, p, p, p,
+                                                 i32]
         _lib = lib
         return lib
 
@@ -273,3 +286,58 @@ def greedy_tokens(logits64):
     t = np.zeros(n, np.int32)
     lib.oracle_greedy_tokens(_ptr(x), n, V, _ptr(t))
     return t
+
+
+def philox4x32_10(counter, key):
+    """Philox4x32-10 of one 4-word counter under a 2-word key (uint32 words)."""
+    lib = _load()
+    c = _c(counter, np.uint32)
+    k = _c(key, np.uint32)
+    if c.shape != (4,) or k.shape != (2,):
+        raise ValueError("counter has 4 words, key 2")
+    out = np.zeros(4, np.uint32)
+    lib.oracle_philox4x32_10(_ptr(c), _ptr(k), _ptr(out))
+    return out
+
+
+def sampled_tokens(logits, temperature: float, seed: int, offset: int,
+                   threads: int | None = None):
+    """Gumbel-max samples of softmax(logits / T) per row (fp64 scores) and each
+    row's margin between the winning score and the runner-up's."""
+    lib = _load()
+    x = np.ascontiguousarray(np.asarray(logits, dtype=np.float32))
+    if x.ndim != 2:
+        raise ValueError("logits must be [R, V]")
+    R, V = x.shape
+    t = np.zeros(R, np.int32)
+    margin = np.zeros(R, np.float64)
+    rc = lib.oracle_sampled_tokens(_ptr(x), V, V, R, float(temperature), int(seed) & (2**64 - 1),
+                                   int(offset) & (2**64 - 1), _ptr(t), _ptr(margin),
+                                   threads or default_threads())
+    if rc != 0:
+        raise ValueError(f"oracle_sampled_tokens: bad input (code {rc})")
+    return t, margin
+
+
+def consensus_sampled(logits, draft_tokens, cu_block, temperature: float, seed: int, offset: int,
+                      threads: int | None = None):
+    """Consensus at temperature T > 0: (accept_len[B], next_token[B], tokens[R])."""
+    lib = _load()
+    x = np.ascontiguousarray(np.asarray(logits, dtype=np.float32))
+    if x.ndim != 2:
+        raise ValueError("logits must be [R, V]")
+    R, V = x.shape
+    dr = _c(draft_tokens, np.int32)
+    cu = _c(cu_block, np.int32)
+    B = cu.shape[0] - 1
+    if dr.shape[0] != R or int(cu[-1]) != R:
+        raise ValueError("inconsistent consensus shapes")
+    acc = np.zeros(B, np.int32)
+    nxt = np.zeros(B, np.int32)
+    t = np.zeros(R, np.int32)
+    rc = lib.oracle_consensus_sampled(_ptr(x), V, V, _ptr(dr), _ptr(cu), B, float(temperature),
+                                      int(seed) & (2**64 - 1), int(offset) & (2**64 - 1),
+                                      _ptr(acc), _ptr(nxt), _ptr(t), threads or default_threads())
+    if rc != 0:
+        raise ValueError(f"oracle_consensus_sampled: bad input (code {rc})")
+    return acc, nxt, t

@@ -499,3 +499,112 @@ void oracle_greedy_tokens(const double* logits, int64_t nrows, int V, int32_t* t
     t[i] = idx;
   }
 }
+
+/* ------------------------------------------------------------------------- */
+/* Temperature > 0 consensus (the pages fix no sampling rule; this is the
+ * reading taken): the frozen AR view's token of row r is a sample from
+ * softmax(logits[r] / T), drawn by the Gumbel-max rule
+ *     t_r = argmax_v ( logits[r, v] / T + g_{r,v} ),   g = -ln(-ln u),
+ * with u_{r,v} in (0, 1) from the counter-based generator Philox4x32-10
+ * (Salmon, Moraes, Dror, Shaw, "Parallel random numbers: as easy as 1, 2, 3",
+ * SC 2011), and a draft is accepted iff it equals that sample, left to right,
+ * exactly as in the greedy rule (technical summary §2.3 item 3). Every
+ * committed token is the AR view's own sample, so the emitted stream is an
+ * AR sample at temperature T. Scores here are in fp64. */
+
+/* One Philox4x32 round and the key schedule, as published. */
+static void philox_round(uint32_t c[4], const uint32_t k[2]) {
+  const uint64_t p0 = (uint64_t)0xD2511F53u * c[0];
+  const uint64_t p1 = (uint64_t)0xCD9E8D57u * c[2];
+  const uint32_t hi0 = (uint32_t)(p0 >> 32), lo0 = (uint32_t)p0;
+  const uint32_t hi1 = (uint32_t)(p1 >> 32), lo1 = (uint32_t)p1;
+  const uint32_t n0 = hi1 ^ c[1] ^ k[0];
+  const uint32_t n2 = hi0 ^ c[3] ^ k[1];
+  c[0] = n0;
+  c[1] = lo1;
+  c[2] = n2;
+  c[3] = lo0;
+}
+
+/* Philox4x32-10: ten rounds, the key bumped by the Weyl constants between
+ * rounds. out may alias ctr. */
+void oracle_philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t out[4]) {
+  uint32_t c[4] = {ctr[0], ctr[1], ctr[2], ctr[3]};
+  uint32_t k[2] = {key[0], key[1]};
+  for (int i = 0; i < 10; ++i) {
+    if (i > 0) {
+      k[0] += 0x9E3779B9u;
+      k[1] += 0xBB67AE85u;
+    }
+    philox_round(c, k);
+  }
+  for (int i = 0; i < 4; ++i) out[i] = c[i];
+}
+
+/* u_{r,v}: word (v mod 4) of Philox4x32-10 at counter (v / 4, r, offset low,
+ * offset high) and key (seed low, seed high); its top 24 bits plus one half,
+ * over 2^24: a value in (0, 1), never 0 or 1. */
+static double sample_uniform(int64_t r, int v, uint64_t seed, uint64_t offset) {
+  const uint32_t ctr[4] = {(uint32_t)(v >> 2), (uint32_t)r, (uint32_t)offset,
+                           (uint32_t)(offset >> 32)};
+  const uint32_t key[2] = {(uint32_t)seed, (uint32_t)(seed >> 32)};
+  uint32_t w[4];
+  oracle_philox4x32_10(ctr, key, w);
+  return ((double)(w[v & 3] >> 8) + 0.5) / 16777216.0;
+}
+
+typedef struct {
+  const float* logits;
+  int64_t ld;
+  int V;
+  double T;
+  uint64_t seed, offset;
+  int32_t* tokens;
+  double* margin;  /* best score minus the runner-up's (may be NULL) */
+} sample_job;
+
+static void sample_row(void* ctx, int64_t r) {
+  sample_job* a = (sample_job*)ctx;
+  const float* x = a->logits + r * a->ld;
+  double best = -INFINITY, second = -INFINITY;
+  int32_t idx = 0;
+  for (int v = 0; v < a->V; ++v) {
+    double xv = (double)x[v];
+    if (isnan(xv)) xv = -INFINITY;
+    const double u = sample_uniform(r, v, a->seed, a->offset);
+    const double s = xv / a->T - log(-log(u));
+    if (s > best) {
+      second = best;
+      best = s;
+      idx = v;
+    } else if (s > second) {
+      second = s;
+    }
+  }
+  a->tokens[r] = idx;
+  if (a->margin) a->margin[r] = best - second;
+}
+
+/* Sampled AR tokens of rows 0 .. R-1 (and each row's winning margin). */
+int oracle_sampled_tokens(const float* logits, int64_t ld, int V, int64_t R, double T,
+                          uint64_t seed, uint64_t offset, int32_t* tokens, double* margin,
+                          int threads) {
+  if (V < 1 || ld < V || R < 0 || !(T > 0.0)) return -1;
+  sample_job a = {logits, ld, V, T, seed, offset, tokens, margin};
+  parallel_for(R, sample_row, &a, threads);
+  return 0;
+}
+
+/* Consensus at temperature T: the sampled tokens, then the greedy rule's
+ * left-to-right acceptance on them. */
+int oracle_consensus_sampled(const float* logits, int64_t ld, int V, const int32_t* draft,
+                             const int32_t* cu_block, int B, double T, uint64_t seed,
+                             uint64_t offset, int32_t* accept_len, int32_t* next_token,
+                             int32_t* tokens, int threads) {
+  if (B < 0) return -1;
+  const int64_t R = (B > 0) ? cu_block[B] : 0;
+  const int rc = oracle_sampled_tokens(logits, ld, V, R, T, seed, offset, tokens, NULL, threads);
+  if (rc) return rc;
+  oracle_accept(tokens, draft, cu_block, B, accept_len, next_token);
+  return 0;
+}
