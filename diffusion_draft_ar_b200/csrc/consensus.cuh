@@ -132,6 +132,123 @@ __global__ void __launch_bounds__(kConsThreads)
   }
 }
 
+// ---------------------------------------------------------------------------
+// Temperature > 0 (the pages name temperature settings but fix no sampling
+// rule; the rule taken): row r's AR token is the Gumbel-max sample
+//   t_r = argmax_v  logits[r, v] / T - ln(-ln u_{r,v})
+// of softmax(logits[r] / T), and the drafts are accepted left to right iff
+// they equal it, as in the greedy rule (the finalize kernel below). u comes
+// from the counter-based generator Philox4x32-10 (Salmon, Moraes, Dror, Shaw,
+// "Parallel random numbers: as easy as 1, 2, 3", SC 2011): counter
+// (v / 4, r, offset lo, offset hi), key (seed lo, seed hi), word v % 4, and
+// u = (top 24 bits + 1/2) / 2^24, in (0, 1).
+
+struct Philox4 {
+  uint32_t x, y, z, w;
+};
+
+// Philox4x32-10: ten rounds, the key bumped by the Weyl constants between
+// rounds (the published definition).
+__device__ __forceinline__ Philox4 philox4x32_10(uint32_t c0, uint32_t c1, uint32_t c2,
+                                                 uint32_t c3, uint32_t k0, uint32_t k1) {
+#pragma unroll
+  for (int i = 0; i < 10; ++i) {
+    if (i > 0) {
+      k0 += 0x9E3779B9u;
+      k1 += 0xBB67AE85u;
+    }
+    const uint32_t hi0 = __umulhi(0xD2511F53u, c0), lo0 = 0xD2511F53u * c0;
+    const uint32_t hi1 = __umulhi(0xCD9E8D57u, c2), lo1 = 0xCD9E8D57u * c2;
+    const uint32_t n0 = hi1 ^ c1 ^ k0;
+    const uint32_t n2 = hi0 ^ c3 ^ k1;
+    c0 = n0;
+    c1 = lo1;
+    c2 = n2;
+    c3 = lo0;
+  }
+  return Philox4{c0, c1, c2, c3};
+}
+
+// -ln(-ln u) for u = (k + 1/2) / 2^24, k = word >> 8. -ln u is taken with
+// the accurate log1pf(-(1 - u)) when u >= 1/2 (1 - u is exact there and -ln u
+// small, where the largest noise values, the likely winners, come from) and
+// from the base-2 logarithm otherwise (|ln u| >= ln 2, relative error ~2^-22).
+__device__ __forceinline__ float gumbel_noise(uint32_t word) {
+  const uint32_t k = word >> 8;
+  const float u = (static_cast<float>(k) + 0.5f) * 5.9604644775390625e-8f;  // 2^-24
+  float e;
+  if (k >= (1u << 23)) {
+    const float v = (static_cast<float>((1u << 24) - k) - 0.5f) * 5.9604644775390625e-8f;
+    e = -log1pf(-v);
+  } else {
+    e = -0.6931471805599453f * __log2f(u);
+  }
+  return -0.6931471805599453f * __log2f(e);
+}
+
+__device__ __forceinline__ void take_sample(float x, float g, float inv_t, int idx, float& best,
+                                            int& bidx) {
+  const float s = fmaf(x, inv_t, g);  // NaN logits give NaN and never win
+  if (s > best) {
+    best = s;
+    bidx = idx;
+  }
+}
+
+// One CTA per (row, 16,384-entry chunk): every thread takes groups of four
+// consecutive entries (one Philox call each), keeps the first index of its
+// largest score, and the CTA reduces the order-preserving keys as the greedy
+// pass does. The chunk start is a multiple of 4, so a group never straddles
+// two counters; its logits are one 16-byte load when the row allows.
+__global__ void __launch_bounds__(kConsThreads)
+    consensus_sample_kernel(const float* __restrict__ logits, long long ld, int V,
+                            const int* __restrict__ cu_block, int B, int max_block, int n_chunks,
+                            unsigned long long* __restrict__ part, float inv_t, uint32_t seed_lo,
+                            uint32_t seed_hi, uint32_t off_lo, uint32_t off_hi) {
+  pdl_launch_dependents();  // the finalize pass may start its launch now
+  const int r = blockIdx.y;
+  const int R = cu_block ? cu_block[B] : B * max_block;
+  if (r >= R) return;
+  const int c = blockIdx.x;
+  const int v0 = c * kConsChunk;
+  const int v1 = min(V, v0 + kConsChunk);
+  const float* row = logits + static_cast<long long>(r) * ld;
+  const bool vec = ((reinterpret_cast<uintptr_t>(row) & 15u) == 0);
+  const float NEG_INF = -__int_as_float(0x7f800000);
+  float best = NEG_INF;
+  int bidx = -1;
+  const int g0 = v0 >> 2, g1 = (v1 + 3) >> 2;
+  for (int g = g0 + static_cast<int>(threadIdx.x); g < g1; g += kConsThreads) {
+    const int v = g << 2;
+    float x[4];
+    if (vec && v + 3 < v1) {
+      const float4 q = ld_nc_f4(row + v);
+      x[0] = q.x, x[1] = q.y, x[2] = q.z, x[3] = q.w;
+    } else {
+#pragma unroll
+      for (int k = 0; k < 4; ++k) x[k] = (v + k < v1) ? row[v + k] : NEG_INF;
+    }
+    const Philox4 w = philox4x32_10(static_cast<uint32_t>(g), static_cast<uint32_t>(r), off_lo,
+                                    off_hi, seed_lo, seed_hi);
+    if (bidx < 0) bidx = v;  // lowest index this thread sees: the tie default
+    take_sample(x[0], gumbel_noise(w.x), inv_t, v, best, bidx);
+    if (v + 1 < v1) take_sample(x[1], gumbel_noise(w.y), inv_t, v + 1, best, bidx);
+    if (v + 2 < v1) take_sample(x[2], gumbel_noise(w.z), inv_t, v + 2, best, bidx);
+    if (v + 3 < v1) take_sample(x[3], gumbel_noise(w.w), inv_t, v + 3, best, bidx);
+  }
+  const int tid = threadIdx.x;
+  unsigned long long key = (bidx >= 0) ? consensus_key(best, static_cast<uint32_t>(bidx)) : 0ull;
+  key = warp_max_u64(key);
+  __shared__ unsigned long long red[kConsThreads / 32];
+  if ((tid & 31) == 0) red[tid >> 5] = key;
+  __syncthreads();
+  if (tid < 32) {
+    key = tid < kConsThreads / 32 ? red[tid] : 0ull;
+    key = warp_max_u64(key);
+    if (tid == 0) part[static_cast<long long>(r) * n_chunks + c] = key;
+  }
+}
+
 __global__ void consensus_finalize_kernel(const unsigned long long* __restrict__ part,
                                           int n_chunks, const int* __restrict__ draft,
                                           const int* __restrict__ cu_block, int B, int max_block,

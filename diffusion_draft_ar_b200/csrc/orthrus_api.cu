@@ -500,6 +500,62 @@ orthrus_status_t orthrus_consensus_commit(const float* verify_logits, int64_t ld
                          next_token, row_argmax, prefix_lens, workspace, workspace_bytes, stream);
 }
 
+orthrus_status_t orthrus_consensus_sampled(const float* verify_logits, int64_t ld, int32_t V,
+                                           const int32_t* draft_tokens, const int32_t* cu_block,
+                                           int32_t B, int32_t max_block, float temperature,
+                                           uint64_t seed, uint64_t offset, int32_t* accept_len,
+                                           int32_t* next_token, int32_t* row_token,
+                                           int32_t* prefix_lens, void* workspace,
+                                           size_t workspace_bytes, void* stream) {
+  NvtxRange r("orthrus_consensus_sampled");
+  if (!(temperature > 0.f) || !std::isfinite(temperature))
+    return fail(ORTHRUS_ERR_INVALID_ARG, "temperature = %g (must be finite and > 0)",
+                static_cast<double>(temperature));
+  const float inv_t = 1.f / temperature;
+  if (!std::isfinite(inv_t))
+    return fail(ORTHRUS_ERR_UNSUPPORTED, "temperature = %g is too small for fp32 scores",
+                static_cast<double>(temperature));
+  if (B < 0) return fail(ORTHRUS_ERR_INVALID_ARG, "B = %d < 0", B);
+  if (V < 1 || ld < V) return fail(ORTHRUS_ERR_INVALID_ARG, "V = %d, ld = %lld", V, (long long)ld);
+  if (max_block < 1) return fail(ORTHRUS_ERR_INVALID_ARG, "max_block = %d", max_block);
+  if (B == 0) return ok();
+  if (!verify_logits || !draft_tokens || !accept_len || !next_token || !workspace)
+    return fail(ORTHRUS_ERR_INVALID_ARG, "a required pointer is NULL");
+  if (!aligned(verify_logits, 4) || !aligned(workspace, 16))
+    return fail(ORTHRUS_ERR_INVALID_ARG, "misaligned logits or workspace");
+  const long long R_max = static_cast<long long>(B) * max_block;
+  if (R_max > 65535) return fail(ORTHRUS_ERR_UNSUPPORTED, "more than 65535 rows");
+  const size_t need = orthrus_consensus_workspace_size(B, max_block, V);
+  if (workspace_bytes < need)
+    return fail(ORTHRUS_ERR_INVALID_ARG, "workspace %zu bytes < %zu needed", workspace_bytes, need);
+  const int n_chunks = (V + kConsChunk - 1) / kConsChunk;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  auto* part = static_cast<unsigned long long*>(workspace);
+  dim3 grid(n_chunks, static_cast<unsigned>(R_max));
+  consensus_sample_kernel<<<grid, kConsThreads, 0, st>>>(
+      verify_logits, ld, V, cu_block, B, max_block, n_chunks, part, inv_t,
+      static_cast<uint32_t>(seed), static_cast<uint32_t>(seed >> 32),
+      static_cast<uint32_t>(offset), static_cast<uint32_t>(offset >> 32));
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(ORTHRUS_ERR_CUDA, "consensus launch: %s", cudaGetErrorString(e));
+  const int warps = 8;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((B + warps - 1) / warps);
+  cfg.blockDim = dim3(warps * 32);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, consensus_finalize_kernel, static_cast<const unsigned long long*>(part),
+                         n_chunks, draft_tokens, cu_block, static_cast<int>(B),
+                         static_cast<int>(max_block), accept_len, next_token, row_token,
+                         prefix_lens, static_cast<int>(R_max));
+  if (e != cudaSuccess) return fail(ORTHRUS_ERR_CUDA, "consensus launch: %s", cudaGetErrorString(e));
+  return ok();
+}
+
 orthrus_status_t orthrus_kv_append(const void* k_block, const void* v_block,
                                    const int32_t* cu_block, int32_t max_block,
                                    const int32_t* accept_len, int32_t* prefix_lens,

@@ -69,6 +69,10 @@ lib.orthrus_lm_head_workspace_size.argtypes = [_i32]
 lib.orthrus_lm_head_consensus.restype = _i32
 lib.orthrus_lm_head_consensus.argtypes = [_vp, _vp, _i32, _i32, _i32, _vp, _vp, _i32, _i32, _vp, _vp,
                                           _vp, _vp, _vp, _sz, _vp, _vp]
+lib.orthrus_consensus_sampled.restype = _i32
+lib.orthrus_consensus_sampled.argtypes = [_vp, _i64, _i32, _vp, _vp, _i32, _i32, _f32,
+                                          ctypes.c_uint64, ctypes.c_uint64, _vp, _vp, _vp, _vp,
+                                          _vp, _sz, _vp]
 lib.orthrus_consensus_noalloc.restype = _i32
 lib.orthrus_consensus_noalloc.argtypes = [_vp, _i64, _i32, _vp, _vp, _i32, _i32, _vp, _vp, _vp, _vp]
 lib.orthrus_status_string.restype = ctypes.c_char_p
@@ -221,6 +225,34 @@ def consensus(verify_logits, draft_tokens, cu_block, B: int, max_block: int, acc
                                _ptr(next_token), _ptr(row_argmax), _ptr(workspace),
                                workspace.numel(), _stream(stream))
     _check(st, "orthrus_consensus")
+
+
+def consensus_sampled(verify_logits, draft_tokens, cu_block, B: int, max_block: int,
+                      temperature: float, seed: int, offset: int, accept_len, next_token,
+                      workspace, row_token=None, prefix_lens=None, stream=None):
+    """``orthrus_consensus_sampled``: consensus at temperature > 0 (Gumbel-max
+    sample of softmax(logits / T) from Philox4x32-10 noise); writes accept_len,
+    next_token (and row_token, and advances prefix_lens when given) in place."""
+    if not verify_logits.is_cuda or verify_logits.dtype != torch.float32 or verify_logits.dim() != 2:
+        raise ValueError("verify_logits must be a 2-D CUDA float32 tensor")
+    if verify_logits.stride(1) != 1:
+        raise ValueError("verify_logits rows must be contiguous")
+    _need(draft_tokens, "draft_tokens", torch.int32, 1)
+    _need(accept_len, "accept_len", torch.int32, 1)
+    _need(next_token, "next_token", torch.int32, 1)
+    _need(workspace, "workspace", torch.uint8)
+    for name, t in (("cu_block", cu_block), ("row_token", row_token),
+                    ("prefix_lens", prefix_lens)):
+        if t is not None:
+            _need(t, name, torch.int32, 1)
+    st = lib.orthrus_consensus_sampled(_ptr(verify_logits), verify_logits.stride(0),
+                                       verify_logits.shape[1], _ptr(draft_tokens), _ptr(cu_block),
+                                       int(B), int(max_block), float(temperature),
+                                       int(seed) & (2 ** 64 - 1), int(offset) & (2 ** 64 - 1),
+                                       _ptr(accept_len), _ptr(next_token), _ptr(row_token),
+                                       _ptr(prefix_lens), _ptr(workspace), workspace.numel(),
+                                       _stream(stream))
+    _check(st, "orthrus_consensus_sampled")
 
 
 def consensus_noalloc(verify_logits, draft_tokens, cu_block, B: int, max_block: int, accept_len,

@@ -22,7 +22,9 @@
  *   orthrus_lm_head_consensus
  *                       the AR model's LM head (hidden states x output
  *                       projection) with the greedy argmax in its epilogue,
- *                       then the consensus rule; the logits are never written.
+ *                       then the consensus rule; the logits are never written;
+ *   orthrus_consensus_sampled
+ *                       consensus at temperature > 0 (a sampled AR token).
  *
  * Conventions shared by every call:
  *   - Every pointer marked "device" is a device pointer owned by the caller; the
@@ -237,6 +239,38 @@ ORTHRUS_API orthrus_status_t orthrus_consensus_commit(const float* verify_logits
                                                       int32_t* next_token, int32_t* row_argmax,
                                                       int32_t* prefix_lens, void* workspace,
                                                       size_t workspace_bytes, void* stream);
+
+/*
+ * Consensus at temperature T > 0. The pages name temperature settings
+ * (technical summary §4) but give no sampling rule; this library's rule keeps
+ * the greedy rule's exact-match acceptance (§2.3 item 3) and replaces the AR
+ * view's greedy token by a sample from softmax(logits / T), drawn with the
+ * Gumbel-max rule. For every block row r:
+ *
+ *   t_r = argmax_v  verify_logits[r, v] / T - ln(-ln u_{r,v})
+ *
+ * (ties to the lowest v, NaN never chosen), where u_{r,v} in (0, 1) is word
+ * v % 4 of Philox4x32-10 (Salmon et al., "Parallel random numbers: as easy as
+ * 1, 2, 3", SC 2011) at counter (v / 4, r, offset & 0xffffffff, offset >> 32)
+ * and key (seed & 0xffffffff, seed >> 32), as (word >> 8) + 1/2 over 2^24.
+ * Then accept_len, next_token (and, when prefix_lens is given, the commit
+ * prefix_lens[b] += accept_len[b]) follow orthrus_consensus's rule on t.
+ * Every committed token is the AR view's own sample, so the emitted stream is
+ * an AR sample at temperature T; give each round a new offset (or seed) so
+ * that no position reuses its noise. Scores are fp32 (logits * (1/T) + noise).
+ *
+ *   temperature  finite, > 0, with 1/T finite in fp32
+ *   row_token    device int32 [R] or NULL: the sampled t_r (written when given)
+ *   prefix_lens  device int32 [B] or NULL (advanced by accept_len when given)
+ *   workspace    as orthrus_consensus (orthrus_consensus_workspace_size)
+ * Other arguments as orthrus_consensus. Errors: as orthrus_consensus, and
+ * INVALID_ARG / UNSUPPORTED for a temperature outside the range above.
+ */
+ORTHRUS_API orthrus_status_t orthrus_consensus_sampled(
+    const float* verify_logits, int64_t ld, int32_t V, const int32_t* draft_tokens,
+    const int32_t* cu_block, int32_t B, int32_t max_block, float temperature, uint64_t seed,
+    uint64_t offset, int32_t* accept_len, int32_t* next_token, int32_t* row_token,
+    int32_t* prefix_lens, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * Fused LM head + greedy consensus (technical summary §2.3 items 2-3 with §2.1:

@@ -232,3 +232,15 @@ def test_lm_head_workspace_size(O):
     assert O.lm_head_workspace_size(512) == 4096
     assert O.lm_head_workspace_size(33) == 512
     assert O.lm_head_workspace_size(0) == 0
+
+
+@pytest.mark.parametrize("T", [0.0, -1.0, float("inf"), float("nan"), 1e-45])
+def test_sampled_consensus_rejects_bad_temperatures_on_the_host(O, T):
+    """Temperature 0, negative, infinite, NaN, or so small that 1/T overflows
+    fp32: refused before any CUDA call."""
+    V = 1000
+    st = O.lib.orthrus_consensus_sampled(ctypes.c_void_p(16), V, V, ctypes.c_void_p(16), None,
+                                         2, 4, T, 1, 2, ctypes.c_void_p(16), ctypes.c_void_p(16),
+                                         None, None, ctypes.c_void_p(16), 1 << 20, None)
+    assert st in (O.ERR_INVALID_ARG, O.ERR_UNSUPPORTED)
+    assert b"temperature" in O.lib.orthrus_last_error()
