@@ -578,6 +578,30 @@ def run_ours(args):
                  "note": "orthrus_kv_append of the accepted VERIFY rows (K and V, read + write), "
                          "prefix lengths restored before each call; latency-bound at this size"}
 
+    # ---- consensus at temperature 1 (Gumbel-max sample) on the same logits
+    s_acc = torch.zeros(m.B, dtype=torch.int32, device=dev)
+    s_nxt = torch.zeros(m.B, dtype=torch.int32, device=dev)
+    s_args = (r.logits.data_ptr(), w.vocab, w.vocab, drafts.data_ptr(), cu.data_ptr(), m.B,
+              w.max_block, 1.0, 1234, 0, s_acc.data_ptr(), s_nxt.data_ptr(), None, None,
+              cons.ws.data_ptr(), cons.ws.numel(), sp)
+
+    def sampled():
+        st = O.lib.orthrus_consensus_sampled(*s_args)
+        if st:
+            raise RuntimeError(f"consensus_sampled failed: {O.lib.orthrus_last_error().decode()}")
+
+    for _ in range(3):
+        scrub(); sampled()
+    t = timed_calls([sampled], 20, scrub, stream)[:, 0]
+    smp_us = float(np.median(t)) * 1e3
+    consensus_sampled = {
+        "us": smp_us, "temperature": 1.0,
+        "gbs": consensus_bytes(w, m) / (smp_us * 1e-6) / 1e9,
+        "rows_per_s": m.R / (smp_us * 1e-6),
+        "vs_greedy": smp_us / (t_cons * 1e3),
+        "note": "orthrus_consensus_sampled: Philox4x32-10 noise and two logarithms per "
+                "logit on the fly (no noise read from memory); ALU-bound"}
+
     # ---- end to end through the public API: pinned host inputs in, results out ----
     e2e_steps = max(1, min(args.steps, args.e2e_steps))
     h_in = {k: t.cpu().pin_memory() for k, t in (
@@ -659,6 +683,7 @@ def run_ours(args):
             "consensus_gbs": consensus_bytes(w, m) / (t_cons * 1e-3) / 1e9,
             "kv_append_us": t_app * 1e3 if t_app is not None else None,
             "kv_append": kv_append,
+            "consensus_sampled": consensus_sampled,
             "commit": ("write-then-truncate (VERIFY attention stores the block K/V; "
                        "consensus advances the lengths)") if write else
                       "separate kv_append of the accepted rows",

@@ -157,8 +157,10 @@ __device__ __forceinline__ Philox4 philox4x32_10(uint32_t c0, uint32_t c1, uint3
       k0 += 0x9E3779B9u;
       k1 += 0xBB67AE85u;
     }
-    const uint32_t hi0 = __umulhi(0xD2511F53u, c0), lo0 = 0xD2511F53u * c0;
-    const uint32_t hi1 = __umulhi(0xCD9E8D57u, c2), lo1 = 0xCD9E8D57u * c2;
+    const uint64_t p0 = static_cast<uint64_t>(0xD2511F53u) * c0;  // one wide multiply each
+    const uint64_t p1 = static_cast<uint64_t>(0xCD9E8D57u) * c2;
+    const uint32_t hi0 = static_cast<uint32_t>(p0 >> 32), lo0 = static_cast<uint32_t>(p0);
+    const uint32_t hi1 = static_cast<uint32_t>(p1 >> 32), lo1 = static_cast<uint32_t>(p1);
     const uint32_t n0 = hi1 ^ c1 ^ k0;
     const uint32_t n2 = hi0 ^ c3 ^ k1;
     c0 = n0;
@@ -169,18 +171,27 @@ __device__ __forceinline__ Philox4 philox4x32_10(uint32_t c0, uint32_t c1, uint3
   return Philox4{c0, c1, c2, c3};
 }
 
-// -ln(-ln u) for u = (k + 1/2) / 2^24, k = word >> 8. -ln u is taken with
-// the accurate log1pf(-(1 - u)) when u >= 1/2 (1 - u is exact there and -ln u
-// small, where the largest noise values, the likely winners, come from) and
-// from the base-2 logarithm otherwise (|ln u| >= ln 2, relative error ~2^-22).
+// -ln(-ln u) for u = (k + 1/2) / 2^24, k = word >> 8. e = -ln u must be
+// accurate in relative terms, since g = -ln e. For u < 15/16, |log2 u| >= 0.09
+// and the hardware base-2 logarithm (absolute error ~2^-22) gives e to ~3e-6.
+// For u >= 15/16 (where the largest noise values, the likely winners, come
+// from) e is the series of -ln(1 - v) = v + v^2/2 + v^3/3 + ... in v = 1 - u,
+// which is exact in fp32; seven terms leave a relative error below v^7/8 <=
+// 2^-31. The outer logarithm needs only absolute accuracy (~2e-7 in g).
 __device__ __forceinline__ float gumbel_noise(uint32_t word) {
   const uint32_t k = word >> 8;
-  const float u = (static_cast<float>(k) + 0.5f) * 5.9604644775390625e-8f;  // 2^-24
   float e;
-  if (k >= (1u << 23)) {
+  if (k >= (15u << 20)) {
     const float v = (static_cast<float>((1u << 24) - k) - 0.5f) * 5.9604644775390625e-8f;
-    e = -log1pf(-v);
+    float q = fmaf(v, 1.f / 7.f, 1.f / 6.f);
+    q = fmaf(v, q, 0.2f);
+    q = fmaf(v, q, 0.25f);
+    q = fmaf(v, q, 1.f / 3.f);
+    q = fmaf(v, q, 0.5f);
+    q = fmaf(v, q, 1.f);
+    e = v * q;
   } else {
+    const float u = (static_cast<float>(k) + 0.5f) * 5.9604644775390625e-8f;  // 2^-24
     e = -0.6931471805599453f * __log2f(u);
   }
   return -0.6931471805599453f * __log2f(e);
