@@ -1103,6 +1103,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     prefetch_tmap(&tm_vc);
     prefetch_tmap(&tm_kb);
     prefetch_tmap(&tm_vb);
+    // Start the cold DRAM reads the first copies depend on while the barriers
+    // and tensor memory are set up: the page-table line of the first tiles
+    // and the first unit's Q tile (into L2; the copies proper follow).
+    const SeqInfo sq = tab.get(a, start.b);
+    const int tiles_per_page = a.page_size / kTileN;
+    if (start.t < (sq.L + kTileN - 1) / kTileN)  // a prefix tile: its page id is in the table
+      prefetch_l2(a.page_table + (long long)start.b * a.max_pages + start.t / tiles_per_page);
+#pragma unroll
+    for (int p = 0; p < Lay::DH; ++p) tma_prefetch_3d(&tm_q, p * 64, start.h * a.G, sq.row0);
   }
   if (warp == kMmaWarp0) {
     tmem_alloc(smem_u32(tmem_slot), kTmemCols);
