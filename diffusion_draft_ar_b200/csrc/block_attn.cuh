@@ -189,8 +189,15 @@ struct SegCursor {
   int b, h, t;
   long long remaining;
   int first;
-  int cta;
+  int cta;  // partial slot: the CTA (balanced, proportional) or the chunk slot (fixed chunks)
 };
+
+// Fixed chunks: slot j is chunk j % max_chunks of unit j / max_chunks. The
+// grid is at most one CTA per SM, and CTA c takes the slots c, c + grid,
+// c + 2 grid, ... that hold tiles, one segment each. Points the cursor at the
+// first such slot at or after j; false (remaining = 0) when there is none.
+__device__ __forceinline__ bool chunk_seek(const AttnArgs& a, const SeqTable& tab, long long j,
+                                           SegCursor& c);
 
 __device__ __forceinline__ bool cursor_next(const AttnArgs& a, const SeqTable& tab, SegCursor& c,
                                             Segment& s) {
@@ -206,6 +213,10 @@ __device__ __forceinline__ bool cursor_next(const AttnArgs& a, const SeqTable& t
   const bool full = (s.t0 == 0 && s.t1 == nt);
   s.part = full ? -1 : (a.chunked ? c.cta : c.cta * 2 + (c.first ? 0 : 1));
   c.first = 0;
+  if (a.chunked == 1) {
+    chunk_seek(a, tab, (long long)c.cta + a.num_ctas, c);
+    return true;
+  }
   c.remaining -= (t1 - c.t);
   c.t = 0;
   if (++c.h == a.Hkv) {
@@ -215,6 +226,29 @@ __device__ __forceinline__ bool cursor_next(const AttnArgs& a, const SeqTable& t
     } while (c.b < a.B && tab.nt(a, c.b) == 0);
   }
   return true;
+}
+
+__device__ __forceinline__ bool chunk_seek(const AttnArgs& a, const SeqTable& tab, long long j,
+                                           SegCursor& c) {
+  const long long slots = (long long)a.B * a.Hkv * a.max_chunks;
+  for (; j < slots; j += a.num_ctas) {
+    const long long u = j / a.max_chunks;
+    const int k = (int)(j - u * a.max_chunks);
+    const int b = (int)(u / a.Hkv);
+    const int nt = tab.nt(a, b);
+    if (nt <= 0) continue;
+    const int nc = unit_chunks(a, nt);
+    if (k >= nc) continue;
+    c.b = b;
+    c.h = (int)(u - (long long)b * a.Hkv);
+    c.t = k * a.chunk_tiles;
+    c.remaining = (k == nc - 1) ? nt - c.t : a.chunk_tiles;
+    c.cta = (int)j;
+    return true;
+  }
+  c.b = a.B;
+  c.remaining = 0;
+  return false;
 }
 
 // ---------------------------------------------------------------------------
@@ -331,7 +365,7 @@ __device__ __forceinline__ bool schedule_prologue(const AttnArgs& a, uint8_t* sm
                                                   SeqTable& tab, SegCursor& start) {
   using Lay = AttnLayout<D>;
   constexpr int kWarps = kAttnThreads / 32;
-  int* sc = reinterpret_cast<int*>(smem + Lay::kSchedOff);  // b, h, t
+  int* sc = reinterpret_cast<int*>(smem + Lay::kSchedOff);  // b, h, t, chunk slot
   long long* srem = reinterpret_cast<long long*>(smem + Lay::kSchedOff + 16);
   long long* scan = reinterpret_cast<long long*>(smem + Lay::kScanOff);
   int4* rows = reinterpret_cast<int4*>(smem + Lay::kSeqOff);
@@ -374,22 +408,10 @@ __device__ __forceinline__ bool schedule_prologue(const AttnArgs& a, uint8_t* sm
     }
   } else if (a.chunked) {
     if (tid == 0) {
-      int b = a.B, h = 0, t = 0;
-      long long rem = 0;
-      const int chunk = blockIdx.x % a.max_chunks;
-      const int u = blockIdx.x / a.max_chunks;
-      const int bu = u / a.Hkv;
-      if (bu < a.B) {
-        const int nt = tab.nt(a, bu);
-        if (nt > 0 && chunk < unit_chunks(a, nt)) {
-          b = bu;
-          h = u % a.Hkv;
-          t = chunk * a.chunk_tiles;
-          rem = (chunk == unit_chunks(a, nt) - 1) ? (nt - t) : a.chunk_tiles;
-        }
-      }
-      sc[0] = b, sc[1] = h, sc[2] = t;
-      *srem = rem;
+      SegCursor c;
+      chunk_seek(a, tab, blockIdx.x, c);
+      sc[0] = c.b, sc[1] = c.h, sc[2] = c.t, sc[3] = c.cta;
+      *srem = c.remaining;
     }
   } else {
     const long long g0 = range_begin(T, blockIdx.x, a.num_ctas);
@@ -432,7 +454,7 @@ __device__ __forceinline__ bool schedule_prologue(const AttnArgs& a, uint8_t* sm
     }
   }
   __syncthreads();
-  start.cta = blockIdx.x;
+  start.cta = a.chunked == 1 ? sc[3] : (int)blockIdx.x;
   start.first = 1;
   start.b = sc[0];
   start.h = sc[1];
@@ -1150,16 +1172,30 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
 // ---------------------------------------------------------------------------
 // Combine: merge the partials of every unit that was cut across CTAs.
-// grid = (B * Hkv, 4 blocks of 32 query rows, 1 or D / 32); 8 warps per CTA,
-// lane = query row. With a third grid dimension of D / 32 (fixed chunks: many
-// partials per unit) each CTA owns 32 columns and its 8 warps split the
-// partials; with 1 (balanced split: two or three partials) the warps split
-// the column blocks and, within each, the partials. Warp 0 finds the unit's partials once per CTA; the
-// partials themselves are read only after the attention grid's writes are
-// visible (griddepcontrol.wait).
+// grid.x: under a chunked schedule one CTA row per (sequence, KV head) unit;
+// under balanced ranges one per boundary between attention CTAs x and x + 1
+// (only a boundary inside a unit cuts it, and the first boundary inside a
+// unit merges it), so no CTA is launched for the many uncut units.
+// grid.y: blocks of 32 query rows; grid.z: column groups. 8 warps per CTA,
+// lane = query row. A CTA covers D / gridDim.z columns in slices of 16, and
+// its warps split over (slice, partial class): warp w takes slice w / wpc and
+// the partials k = w % wpc, w % wpc + wpc, ... (wpc warps per slice). Warp 0
+// finds the unit and its partials once per CTA, before griddepcontrol.wait,
+// so this overlaps the attention grid's tail.
+//
+// The reads are latency-bound (a few KB per warp), so a warp issues the loads
+// of kBatch partials (log-sum-exp and 16 columns each) together, one round
+// trip per batch, and keeps its own running (max, sum, accumulator); the warps
+// of a slice are then merged in shared memory with the same log-sum-exp
+// identity: O = sum_k 2^(lse_k - M) O_k / sum_k 2^(lse_k - M). Chunked
+// schedules use batches of 4 (many partials per unit); balanced ranges leave
+// two or three partials per cut unit and use batches of 2, which keeps the
+// kernel at 64 registers: four CTAs per SM wait at griddepcontrol.wait
+// instead of two.
 
 constexpr int kCombineWarps = 8;
 constexpr int kCombineThreads = 32 * kCombineWarps;
+constexpr int kCombineSlice = 16;  // columns per warp
 
 __device__ __forceinline__ int cta_of_tile(long long T, int C, long long t) {
   long long c = ((t + 1) * C - 1) / T;
@@ -1169,26 +1205,30 @@ __device__ __forceinline__ int cta_of_tile(long long T, int C, long long t) {
   return (int)c;
 }
 
-template <int D>
-__global__ void __launch_bounds__(kCombineThreads)
+template <int D, int kBatch>
+__global__ void __launch_bounds__(kCombineThreads, kBatch == 2 ? 4 : 1)
     attn_combine_kernel(const AttnArgs a) {
   __shared__ long long sh_T, sh_su;
-  __shared__ int sh_clo, sh_count, sh_skip;
+  __shared__ int sh_b, sh_h, sh_clo, sh_count, sh_skip;
   __shared__ float sh_m[kCombineWarps][32];
-  __shared__ float sh_w[kCombineWarps][32];
-  __shared__ float sh_acc[kCombineWarps][32][33];
-  const int u = blockIdx.x, rb = blockIdx.y;
-  const int b = u / a.Hkv, h = u % a.Hkv;
+  __shared__ float sh_l[kCombineWarps][32];
+  __shared__ float sh_acc[kCombineWarps][32][kCombineSlice + 1];
+  const int rb = blockIdx.y;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int Kb = (b < a.B) ? seq_block_len(a, b) : 0;
-  const int rows_valid = a.G * Kb;
-  if (Kb <= 0 || rb * 32 >= rows_valid) return;
-  const int nt = seq_tiles(a, b);
+  if (a.chunked) {
+    // the unit is the CTA row; a unit without rows in this row block has nothing to merge
+    const int b = blockIdx.x / a.Hkv;
+    const int Kb = (b < a.B) ? seq_block_len(a, b) : 0;
+    if (Kb <= 0 || rb * 32 >= a.G * Kb) return;
+  }
   if (warp == 0) {
-    int skip = 0, count = 0, c_lo = 0;
+    int skip = 1, count = 0, c_lo = 0, b = 0, h = 0;
     long long T = 0, s_u = 0;
     if (a.chunked == 2) {
       // the attention kernel's allocation: T, U, then the CTAs of sequences < b
+      b = blockIdx.x / a.Hkv;
+      h = blockIdx.x % a.Hkv;
+      const int nt = seq_tiles(a, b);
       long long t_part = 0;
       int u_part = 0;
       for (int bb = lane; bb < a.B; bb += 32) {
@@ -1210,31 +1250,61 @@ __global__ void __launch_bounds__(kCombineThreads)
       c_lo = (int)(before + (long long)h * count);  // first part (= CTA) of this unit
       skip = count <= 1;
     } else if (a.chunked) {
-      count = unit_chunks(a, nt);
+      b = blockIdx.x / a.Hkv;
+      h = blockIdx.x % a.Hkv;
+      count = unit_chunks(a, seq_tiles(a, b));
       skip = count <= 1;
     } else {
-      // total tiles and this unit's first tile, summed across the warp
-      long long t_part = 0, s_part = 0;
-      for (int bb = lane; bb < a.B; bb += 32) {
-        const long long n = (long long)a.Hkv * seq_tiles(a, bb);
-        t_part += n;
-        if (bb < b) s_part += n;
-      }
+      // total tiles, then the unit holding the boundary tile g (the first
+      // tile of attention CTA x + 1), found by a scan over the sequences
+      const int C = a.num_ctas, x = blockIdx.x;
+      long long t_part = 0;
+      for (int bb = lane; bb < a.B; bb += 32) t_part += (long long)a.Hkv * seq_tiles(a, bb);
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        t_part += __shfl_xor_sync(0xffffffffu, t_part, o);
-        s_part += __shfl_xor_sync(0xffffffffu, s_part, o);
-      }
+      for (int o = 16; o > 0; o >>= 1) t_part += __shfl_xor_sync(0xffffffffu, t_part, o);
       T = t_part;
-      s_u = s_part + (long long)h * nt;
-      c_lo = cta_of_tile(T, a.num_ctas, s_u);
-      const int c_hi = cta_of_tile(T, a.num_ctas, s_u + nt - 1);
-      skip = c_lo == c_hi;
-      count = c_hi - c_lo + 1;
+      const long long g = T > 0 ? range_begin(T, x + 1, C) : 0;
+      long long base = 0, s_b = -1;
+      int nt = 0;
+      for (int b0 = 0; g < T && b0 < a.B; b0 += 32) {
+        const int bb = b0 + lane;
+        const int n_t = bb < a.B ? seq_tiles(a, bb) : 0;
+        const long long n = (long long)a.Hkv * n_t;
+        long long incl = n;  // inclusive scan within the warp
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const long long y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += y;
+        }
+        const long long excl = base + incl - n;
+        const unsigned hit = __ballot_sync(0xffffffffu, n > 0 && excl <= g && g < excl + n);
+        if (hit) {
+          const int src = __ffs(hit) - 1;
+          s_b = __shfl_sync(0xffffffffu, excl, src);
+          nt = __shfl_sync(0xffffffffu, n_t, src);
+          b = b0 + src;
+          break;
+        }
+        base += __shfl_sync(0xffffffffu, incl, 31);
+      }
+      if (s_b >= 0) {
+        h = (int)((g - s_b) / nt);
+        const long long t = g - s_b - (long long)h * nt;
+        s_u = s_b + (long long)h * nt;
+        c_lo = cta_of_tile(T, C, s_u);
+        // a cut (not a unit start), merged by the first boundary inside the unit
+        if (t != 0 && c_lo == x) {
+          const int c_hi = cta_of_tile(T, C, s_u + nt - 1);
+          count = c_hi - c_lo + 1;
+          skip = 0;
+        }
+      }
     }
     if (lane == 0) {
       sh_T = T;
       sh_su = s_u;
+      sh_b = b;
+      sh_h = h;
       sh_clo = c_lo;
       sh_count = count;
       sh_skip = skip;
@@ -1242,8 +1312,14 @@ __global__ void __launch_bounds__(kCombineThreads)
   }
   __syncthreads();
   if (sh_skip) return;
+  const int b = sh_b, h = sh_h;
+  const int Kb = seq_block_len(a, b);
+  const int rows_valid = a.G * Kb;
+  if (Kb <= 0 || rb * 32 >= rows_valid) return;
+  const int row0 = seq_row0(a, b);
   const long long T = sh_T, s_u = sh_su;
   const int c_lo = sh_clo, count = sh_count;
+  const int u = b * a.Hkv + h;
 
   auto part_of = [&](int k, bool& use) -> int {
     if (a.chunked == 2) {
@@ -1261,61 +1337,75 @@ __global__ void __launch_bounds__(kCombineThreads)
     return cc * 2 + slot;
   };
 
-  pdl_wait();  // partials written by the attention grid are visible from here on
+  const int cols = D / gridDim.z;           // columns of this CTA
+  const int ncs = cols / kCombineSlice;     // slices
+  const int wpc = kCombineWarps / ncs;      // warps per slice
+  const int sl = warp / wpc, kw = warp % wpc;
+  const int c0 = blockIdx.z * cols + sl * kCombineSlice;
   const int r = rb * 32 + lane;  // query row of this lane (rows past rows_valid are ignored)
   const float NEG_INF = -__int_as_float(0x7f800000);
-  // 1. the row's maximum log-sum-exp over all partials
-  float M = NEG_INF;
-  for (int k = warp; k < count; k += kCombineWarps) {
-    bool use;
-    const int p = part_of(k, use);
-    if (use) M = fmaxf(M, a.ws_lse[(long long)p * kTileM + r]);
+
+  pdl_wait();  // partials written by the attention grid are visible from here on
+  float m_run = NEG_INF, l_run = 0.f;
+  float acc[kCombineSlice];
+#pragma unroll
+  for (int e = 0; e < kCombineSlice; ++e) acc[e] = 0.f;
+  for (int k0 = kw; k0 < count; k0 += wpc * kBatch) {
+    float lse[kBatch];
+    float x[kBatch][kCombineSlice];
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j) {
+      const int k = k0 + j * wpc;
+      bool use = false;
+      const int p = k < count ? part_of(k, use) : 0;
+      lse[j] = use ? a.ws_lse[(long long)p * kTileM + r] : NEG_INF;
+      const float* src = a.ws_o + part_o<D>(use ? p : 0, r, c0);
+#pragma unroll
+      for (int e = 0; e < kCombineSlice; ++e) x[j][e] = use ? src[32 * e] : 0.f;
+    }
+    float mb = m_run;
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j) mb = fmaxf(mb, lse[j]);
+    if (mb != NEG_INF) {
+      const float sr = exp2f(m_run - mb);  // 0 while nothing is accumulated
+      l_run *= sr;
+#pragma unroll
+      for (int e = 0; e < kCombineSlice; ++e) acc[e] *= sr;
+#pragma unroll
+      for (int j = 0; j < kBatch; ++j) {
+        const float wj = exp2f(lse[j] - mb);
+        l_run += wj;
+#pragma unroll
+        for (int e = 0; e < kCombineSlice; ++e) acc[e] = fmaf(wj, x[j][e], acc[e]);
+      }
+      m_run = mb;
+    }
   }
-  sh_m[warp][lane] = M;
+  sh_m[warp][lane] = m_run;
+  sh_l[warp][lane] = l_run;
+#pragma unroll
+  for (int e = 0; e < kCombineSlice; ++e) sh_acc[warp][lane][e] = acc[e];
   __syncthreads();
-#pragma unroll
-  for (int k = 0; k < kCombineWarps; ++k) M = fmaxf(M, sh_m[k][lane]);
-  // 2. warps split over (column block, partial class): the CTA covers
-  // ncb = (D / 32) / gridDim.z column blocks, wpc = 8 / ncb warps per block;
-  // warp w takes column block blockIdx.z + (w / wpc) * gridDim.z and the
-  // partials k = w % wpc, w % wpc + wpc, ...
-  const int ncb = (D / 32) / gridDim.z;
-  const int wpc = kCombineWarps / ncb;
-  const int cb = blockIdx.z + (warp / wpc) * gridDim.z;
-  const int kw = warp % wpc;
-  float acc[32];
-#pragma unroll
-  for (int e = 0; e < 32; ++e) acc[e] = 0.f;
-  float wsum = 0.f;
-  for (int k = kw; k < count; k += wpc) {
-    bool use;
-    const int p = part_of(k, use);
-    if (!use) continue;
-    const float wgt = exp2f(a.ws_lse[(long long)p * kTileM + r] - M);
-    wsum += wgt;
-    const float* src = a.ws_o + part_o<D>(p, r, cb * 32);
-#pragma unroll
-    for (int e = 0; e < 32; ++e) acc[e] = fmaf(wgt, src[32 * e], acc[e]);
-  }
-  sh_w[warp][lane] = wsum;
-#pragma unroll
-  for (int e = 0; e < 32; ++e) sh_acc[warp][lane][e] = acc[e];
-  __syncthreads();
-  // 3. reduce each column block's wpc warps: thread -> (block, row, column pair)
-  const int row0 = seq_row0(a, b);
-  for (int idx = tid; idx < ncb * 32 * 16; idx += kCombineThreads) {
-    const int j = idx / (32 * 16), rr = (idx >> 4) & 31, e = (idx & 15) * 2;
+  // merge the wpc warps of each slice: thread -> (slice, row, column pair)
+  constexpr int kPairs = kCombineSlice / 2;
+  for (int idx = tid; idx < ncs * 32 * kPairs; idx += kCombineThreads) {
+    const int e = (idx % kPairs) * 2, rr = (idx / kPairs) % 32, s = idx / (32 * kPairs);
     const int q = rb * 32 + rr;
     if (q >= rows_valid) continue;
-    float w = 0.f, x0 = 0.f, x1 = 0.f;
-    for (int k = j * wpc; k < (j + 1) * wpc; ++k) {
-      w += sh_w[k][rr];
-      x0 += sh_acc[k][rr][e];
-      x1 += sh_acc[k][rr][e + 1];
+    float M = NEG_INF;
+    for (int k = s * wpc; k < (s + 1) * wpc; ++k) M = fmaxf(M, sh_m[k][rr]);
+    float l = 0.f, x0 = 0.f, x1 = 0.f;
+    if (M != NEG_INF) {
+      for (int k = s * wpc; k < (s + 1) * wpc; ++k) {
+        const float w = exp2f(sh_m[k][rr] - M);
+        l = fmaf(w, sh_l[k][rr], l);
+        x0 = fmaf(w, sh_acc[k][rr][e], x0);
+        x1 = fmaf(w, sh_acc[k][rr][e + 1], x1);
+      }
     }
-    const float inv = 1.f / w;
+    const float inv = l > 0.f ? 1.f / l : 0.f;
     const int i = q / a.G, g = q - i * a.G;
-    const int c = (blockIdx.z + j * gridDim.z) * 32 + e;
+    const int c = blockIdx.z * cols + s * kCombineSlice + e;
     __nv_bfloat16* dst = a.out + ((long long)(row0 + i) * a.Hq + h * a.G + g) * D + c;
     *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(x0 * inv, x1 * inv);
   }

@@ -192,16 +192,28 @@ orthrus_status_t plan_attn(const orthrus_attn_params* p, int sms, AttnPlan* pl) 
                 pl->R_max);
   const long long max_tokens = static_cast<long long>(p->max_pages_per_seq) * p->page_size;
   if (p->kv_split_tokens > 0) {
+    // Fixed chunks: one partial slot per (unit, chunk). The grid is at most
+    // one CTA per SM (or max_ctas), each walking the slots c, c + grid, ...,
+    // so the chunks beyond the first wave run in CTAs already set up instead
+    // of in a tail of short-lived CTAs.
     pl->chunked = 1;
     pl->chunk_tiles = p->kv_split_tokens / kTileN;
     const long long ptiles = (max_tokens + kTileN - 1) / kTileN;
     long long mc = (ptiles + pl->chunk_tiles - 1) / pl->chunk_tiles;
     if (mc < 1) mc = 1;
-    const long long grid = mc * p->Hkv * static_cast<long long>(p->B);
-    if (grid >= (1ll << 31)) return fail(ORTHRUS_ERR_UNSUPPORTED, "too many chunks");
+    const long long slots = mc * p->Hkv * static_cast<long long>(p->B);
+    if (slots >= (1ll << 31)) return fail(ORTHRUS_ERR_UNSUPPORTED, "too many chunks");
     pl->max_chunks = static_cast<int>(mc);
-    pl->grid = static_cast<int>(grid);
-    pl->parts = pl->grid;
+    // With max_ctas = 0 the slots are spread evenly over as few CTAs as give
+    // the same number of slots per CTA as one per SM would (520 slots on 148
+    // SMs: 4 each over 130 CTAs rather than 3 or 4 over 148).
+    long long cap = p->max_ctas > 0 ? p->max_ctas : std::max(sms, 1);
+    if (p->max_ctas == 0 && slots > cap) {
+      const long long per = (slots + cap - 1) / cap;
+      cap = (slots + per - 1) / per;
+    }
+    pl->grid = static_cast<int>(std::min(slots, cap));
+    pl->parts = static_cast<int>(slots);
     pl->combine = true;
   } else if (p->max_ctas == 0 && static_cast<long long>(p->B) * p->Hkv >= (3LL * sms) / 4 &&
              static_cast<long long>(p->B) * p->Hkv <= sms) {
@@ -337,10 +349,13 @@ orthrus_status_t launch_attn(const orthrus_attn_params* p, const AttnPlan& pl, i
   // tail, and it reads the partials only after griddepcontrol.wait.
   const int row_blocks = (pl.G * p->max_block + 31) / 32;
   cudaLaunchConfig_t cfg = {};
-  // Fixed chunks leave many partials per unit: spread a row block's columns
-  // over D / 32 CTAs. A balanced split leaves two or three: one CTA per row
-  // block is enough.
-  cfg.gridDim = dim3(p->B * p->Hkv, row_blocks, pl.chunked ? D / 32 : 1);
+  // Chunked schedules: one CTA row per unit and one CTA per 16 columns of a
+  // row block (many partials per unit). Balanced ranges: one CTA row per
+  // boundary between attention CTAs (two or three partials per cut unit),
+  // one CTA per row block, its warps on different columns.
+  const bool chunked = pl.chunked != 0;
+  cfg.gridDim = chunked ? dim3(p->B * p->Hkv, row_blocks, D / kCombineSlice)
+                        : dim3(std::max(pl.grid - 1, 1), row_blocks, 1);
   cfg.blockDim = dim3(kCombineThreads);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = stream;
@@ -349,7 +364,8 @@ orthrus_status_t launch_attn(const orthrus_attn_params* p, const AttnPlan& pl, i
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, attn_combine_kernel<D>, a);
+  e = chunked ? cudaLaunchKernelEx(&cfg, attn_combine_kernel<D, 4>, a)
+              : cudaLaunchKernelEx(&cfg, attn_combine_kernel<D, 2>, a);
   if (e != cudaSuccess) return fail(ORTHRUS_ERR_CUDA, "combine launch: %s", cudaGetErrorString(e));
   return ok();
 }
@@ -394,7 +410,7 @@ static orthrus_status_t block_attn_entry(const orthrus_attn_params* p, void* str
     return fail(ORTHRUS_ERR_INVALID_ARG, "empty page table or cache");
   int sms = 0;
   int dev = 0;
-  if (p->kv_split_tokens == 0 && p->max_ctas == 0) {
+  if (p->max_ctas == 0) {
     dev = device_sm_count(&sms);
     if (dev < 0) return fail(ORTHRUS_ERR_CUDA, "no current CUDA device");
   } else {

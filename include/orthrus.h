@@ -132,13 +132,16 @@ typedef struct {
   const int32_t* page_table; /* device [B, max_pages_per_seq] */
   float softmax_scale;       /* <= 0: 1/sqrt(D) */
   int32_t kv_split_tokens;   /* 0: the library's schedule (see max_ctas); > 0: fixed chunks
-                                of this many prefix tokens (a multiple of 64), one CTA each */
+                                of this many prefix tokens (a multiple of 64), each merged
+                                as one partial; at most one CTA per SM (or max_ctas > 0
+                                CTAs) walks the chunks, chunk j in CTA j mod grid */
   int32_t max_ctas;          /* 0: library picks: one CTA per (sequence, KV head) unit
                                 when the units number between 3/4 of the SM count and
                                 the SM count; fewer units: every unit gets SMs in
                                 proportion to its tiles, in near-equal chunks (long
                                 contexts); more units than SMs: a balanced split over
-                                one CTA per SM; > 0: balanced split over this many CTAs */
+                                one CTA per SM; > 0: balanced split over this many CTAs
+                                (with kv_split_tokens > 0: the chunk walkers' grid) */
   void* out;                 /* device bf16 [R, Hq, D] */
   void* workspace;           /* device scratch, >= orthrus_block_attn_workspace_size() bytes,
                                 256-byte aligned; contents need no initialisation */

@@ -57,6 +57,15 @@ def test_ragged_fixed_chunks(view, split):
 
 
 @pytest.mark.parametrize("view", VIEWS)
+@pytest.mark.parametrize("split,max_ctas", [(64, 1), (128, 2), (192, 5), (64, 7)])
+def test_ragged_fixed_chunks_few_walkers(view, split, max_ctas):
+    """Fixed chunks walked by fewer CTAs than chunk slots: CTA c takes slots c,
+    c + grid, ... across units and sequences of different lengths, skipping
+    the slots past a unit's last chunk; every chunk is merged as one partial."""
+    _full_parity(_ragged(seed=2), view, kv_split=split, max_ctas=max_ctas)
+
+
+@pytest.mark.parametrize("view", VIEWS)
 def test_edge_prefix_lengths(view):
     """L in {0, 1, 63, 64, 65, 127, 128} with K in {1, 32}."""
     w = small_workload(name="edges", B=7, Hq=8, Hkv=2, D=128, page_size=64, prefix_len=None,
