@@ -196,7 +196,7 @@ struct SegCursor {
 // grid is at most one CTA per SM, and CTA c takes the slots c, c + grid,
 // c + 2 grid, ... that hold tiles, one segment each. Points the cursor at the
 // first such slot at or after j; false (remaining = 0) when there is none.
-__device__ __forceinline__ bool chunk_seek(const AttnArgs& a, const SeqTable& tab, long long j,
+__device__ __forceinline__ bool chunk_seek(const AttnArgs& a, const SeqTable& tab, int j,
                                            SegCursor& c);
 
 __device__ __forceinline__ bool cursor_next(const AttnArgs& a, const SeqTable& tab, SegCursor& c,
@@ -214,7 +214,7 @@ __device__ __forceinline__ bool cursor_next(const AttnArgs& a, const SeqTable& t
   s.part = full ? -1 : (a.chunked ? c.cta : c.cta * 2 + (c.first ? 0 : 1));
   c.first = 0;
   if (a.chunked == 1) {
-    chunk_seek(a, tab, (long long)c.cta + a.num_ctas, c);
+    chunk_seek(a, tab, c.cta + a.num_ctas, c);
     return true;
   }
   c.remaining -= (t1 - c.t);
@@ -228,22 +228,23 @@ __device__ __forceinline__ bool cursor_next(const AttnArgs& a, const SeqTable& t
   return true;
 }
 
-__device__ __forceinline__ bool chunk_seek(const AttnArgs& a, const SeqTable& tab, long long j,
+// The host keeps the slot count below 2^31 - 2^16, so 32-bit arithmetic holds.
+__device__ __forceinline__ bool chunk_seek(const AttnArgs& a, const SeqTable& tab, int j,
                                            SegCursor& c) {
-  const long long slots = (long long)a.B * a.Hkv * a.max_chunks;
+  const int slots = a.B * a.Hkv * a.max_chunks;
   for (; j < slots; j += a.num_ctas) {
-    const long long u = j / a.max_chunks;
-    const int k = (int)(j - u * a.max_chunks);
-    const int b = (int)(u / a.Hkv);
+    const int u = j / a.max_chunks;
+    const int k = j - u * a.max_chunks;
+    const int b = u / a.Hkv;
     const int nt = tab.nt(a, b);
     if (nt <= 0) continue;
     const int nc = unit_chunks(a, nt);
     if (k >= nc) continue;
     c.b = b;
-    c.h = (int)(u - (long long)b * a.Hkv);
+    c.h = u - b * a.Hkv;
     c.t = k * a.chunk_tiles;
     c.remaining = (k == nc - 1) ? nt - c.t : a.chunk_tiles;
-    c.cta = (int)j;
+    c.cta = j;
     return true;
   }
   c.b = a.B;
@@ -409,7 +410,7 @@ __device__ __forceinline__ bool schedule_prologue(const AttnArgs& a, uint8_t* sm
   } else if (a.chunked) {
     if (tid == 0) {
       SegCursor c;
-      chunk_seek(a, tab, blockIdx.x, c);
+      chunk_seek(a, tab, (int)blockIdx.x, c);
       sc[0] = c.b, sc[1] = c.h, sc[2] = c.t, sc[3] = c.cta;
       *srem = c.remaining;
     }

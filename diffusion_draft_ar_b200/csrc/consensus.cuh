@@ -178,39 +178,36 @@ __device__ __forceinline__ Philox4 philox4x32_10(uint32_t c0, uint32_t c1, uint3
 // from) e is the series of -ln(1 - v) = v + v^2/2 + v^3/3 + ... in v = 1 - u,
 // which is exact in fp32; seven terms leave a relative error below v^7/8 <=
 // 2^-31. The outer logarithm needs only absolute accuracy (~2e-7 in g).
+// Both forms are evaluated and one is selected: in nearly every warp some
+// lane needs the series, so a branch would run both anyway, converting k
+// twice (one conversion here; v = 2^24 - k - 1/2 is exact for the series
+// lanes).
 __device__ __forceinline__ float gumbel_noise(uint32_t word) {
   const uint32_t k = word >> 8;
-  float e;
-  if (k >= (15u << 20)) {
-    const float v = (static_cast<float>((1u << 24) - k) - 0.5f) * 5.9604644775390625e-8f;
-    float q = fmaf(v, 1.f / 7.f, 1.f / 6.f);
-    q = fmaf(v, q, 0.2f);
-    q = fmaf(v, q, 0.25f);
-    q = fmaf(v, q, 1.f / 3.f);
-    q = fmaf(v, q, 0.5f);
-    q = fmaf(v, q, 1.f);
-    e = v * q;
-  } else {
-    const float u = (static_cast<float>(k) + 0.5f) * 5.9604644775390625e-8f;  // 2^-24
-    e = -0.6931471805599453f * __log2f(u);
-  }
+  const float kf = static_cast<float>(k);
+  const float v = ((16777216.f - kf) - 0.5f) * 5.9604644775390625e-8f;  // 2^-24
+  float q = fmaf(v, 1.f / 7.f, 1.f / 6.f);
+  q = fmaf(v, q, 0.2f);
+  q = fmaf(v, q, 0.25f);
+  q = fmaf(v, q, 1.f / 3.f);
+  q = fmaf(v, q, 0.5f);
+  q = fmaf(v, q, 1.f);
+  const float e_series = v * q;
+  const float u = (kf + 0.5f) * 5.9604644775390625e-8f;
+  const float e_log = -0.6931471805599453f * __log2f(u);
+  const float e = (k >= (15u << 20)) ? e_series : e_log;
   return -0.6931471805599453f * __log2f(e);
-}
-
-__device__ __forceinline__ void take_sample(float x, float g, float inv_t, int idx, float& best,
-                                            int& bidx) {
-  const float s = fmaf(x, inv_t, g);  // NaN logits give NaN and never win
-  if (s > best) {
-    best = s;
-    bidx = idx;
-  }
 }
 
 // One CTA per (row, 16,384-entry chunk): every thread takes groups of four
 // consecutive entries (one Philox call each), keeps the first index of its
 // largest score, and the CTA reduces the order-preserving keys as the greedy
 // pass does. The chunk start is a multiple of 4, so a group never straddles
-// two counters; its logits are one 16-byte load when the row allows.
+// two counters; its logits are one 16-byte load when the row allows. Entries
+// past the row end score -inf. A group is compared once, by its largest
+// score m (fmaxf drops NaN, so a NaN logit never wins): only when m beats the
+// thread's best is the first entry equal to m looked up, which keeps the
+// first index of the largest score as a comparison per entry would.
 __global__ void __launch_bounds__(kConsThreads)
     consensus_sample_kernel(const float* __restrict__ logits, long long ld, int V,
                             const int* __restrict__ cu_block, int B, int max_block, int n_chunks,
@@ -242,10 +239,16 @@ __global__ void __launch_bounds__(kConsThreads)
     const Philox4 w = philox4x32_10(static_cast<uint32_t>(g), static_cast<uint32_t>(r), off_lo,
                                     off_hi, seed_lo, seed_hi);
     if (bidx < 0) bidx = v;  // lowest index this thread sees: the tie default
-    take_sample(x[0], gumbel_noise(w.x), inv_t, v, best, bidx);
-    if (v + 1 < v1) take_sample(x[1], gumbel_noise(w.y), inv_t, v + 1, best, bidx);
-    if (v + 2 < v1) take_sample(x[2], gumbel_noise(w.z), inv_t, v + 2, best, bidx);
-    if (v + 3 < v1) take_sample(x[3], gumbel_noise(w.w), inv_t, v + 3, best, bidx);
+    float sc[4];
+    sc[0] = fmaf(x[0], inv_t, gumbel_noise(w.x));
+    sc[1] = fmaf(x[1], inv_t, gumbel_noise(w.y));
+    sc[2] = fmaf(x[2], inv_t, gumbel_noise(w.z));
+    sc[3] = fmaf(x[3], inv_t, gumbel_noise(w.w));
+    const float m = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3]));
+    if (m > best) {
+      best = m;
+      bidx = sc[0] == m ? v : (sc[1] == m ? v + 1 : (sc[2] == m ? v + 2 : v + 3));
+    }
   }
   const int tid = threadIdx.x;
   unsigned long long key = (bidx >= 0) ? consensus_key(best, static_cast<uint32_t>(bidx)) : 0ull;

@@ -202,7 +202,7 @@ orthrus_status_t plan_attn(const orthrus_attn_params* p, int sms, AttnPlan* pl) 
     long long mc = (ptiles + pl->chunk_tiles - 1) / pl->chunk_tiles;
     if (mc < 1) mc = 1;
     const long long slots = mc * p->Hkv * static_cast<long long>(p->B);
-    if (slots >= (1ll << 31)) return fail(ORTHRUS_ERR_UNSUPPORTED, "too many chunks");
+    if (slots >= (1ll << 31) - (1ll << 16)) return fail(ORTHRUS_ERR_UNSUPPORTED, "too many chunks");
     pl->max_chunks = static_cast<int>(mc);
     // With max_ctas = 0 the slots are spread evenly over as few CTAs as give
     // the same number of slots per CTA as one per SM would (520 slots on 148
@@ -212,6 +212,7 @@ orthrus_status_t plan_attn(const orthrus_attn_params* p, int sms, AttnPlan* pl) 
       const long long per = (slots + cap - 1) / cap;
       cap = (slots + per - 1) / per;
     }
+    cap = std::min(cap, 65535LL);  // the walkers' stride: j + grid stays below 2^31
     pl->grid = static_cast<int>(std::min(slots, cap));
     pl->parts = static_cast<int>(slots);
     pl->combine = true;
