@@ -199,6 +199,10 @@ struct SegCursor {
 __device__ __forceinline__ bool chunk_seek(const AttnArgs& a, const SeqTable& tab, int j,
                                            SegCursor& c);
 
+// kWalk: the kernel variant whose CTAs walk several fixed-chunk slots. The
+// other variant runs every schedule in which a fixed-chunk CTA holds one slot
+// (the one-CTA-per-unit plan among them) without the walk's code.
+template <bool kWalk>
 __device__ __forceinline__ bool cursor_next(const AttnArgs& a, const SeqTable& tab, SegCursor& c,
                                             Segment& s) {
   if (c.remaining <= 0 || c.b >= a.B) return false;
@@ -213,7 +217,7 @@ __device__ __forceinline__ bool cursor_next(const AttnArgs& a, const SeqTable& t
   const bool full = (s.t0 == 0 && s.t1 == nt);
   s.part = full ? -1 : (a.chunked ? c.cta : c.cta * 2 + (c.first ? 0 : 1));
   c.first = 0;
-  if (a.chunked == 1) {
+  if (kWalk && a.chunked == 1) {
     chunk_seek(a, tab, c.cta + a.num_ctas, c);
     return true;
   }
@@ -361,7 +365,7 @@ __device__ __forceinline__ long long block_sum_ll(long long x, long long* scan) 
   return t;
 }
 
-template <int D>
+template <int D, bool kWalk>
 __device__ __forceinline__ bool schedule_prologue(const AttnArgs& a, uint8_t* smem,
                                                   SeqTable& tab, SegCursor& start) {
   using Lay = AttnLayout<D>;
@@ -409,10 +413,29 @@ __device__ __forceinline__ bool schedule_prologue(const AttnArgs& a, uint8_t* sm
     }
   } else if (a.chunked) {
     if (tid == 0) {
-      SegCursor c;
-      chunk_seek(a, tab, (int)blockIdx.x, c);
-      sc[0] = c.b, sc[1] = c.h, sc[2] = c.t, sc[3] = c.cta;
-      *srem = c.remaining;
+      if (kWalk) {
+        SegCursor c;
+        chunk_seek(a, tab, (int)blockIdx.x, c);
+        sc[0] = c.b, sc[1] = c.h, sc[2] = c.t, sc[3] = c.cta;
+        *srem = c.remaining;
+      } else {  // one slot per CTA: slot = CTA
+        int b = a.B, h = 0, t = 0;
+        long long rem = 0;
+        const int chunk = blockIdx.x % a.max_chunks;
+        const int u = blockIdx.x / a.max_chunks;
+        const int bu = u / a.Hkv;
+        if (bu < a.B) {
+          const int nt = tab.nt(a, bu);
+          if (nt > 0 && chunk < unit_chunks(a, nt)) {
+            b = bu;
+            h = u % a.Hkv;
+            t = chunk * a.chunk_tiles;
+            rem = (chunk == unit_chunks(a, nt) - 1) ? (nt - t) : a.chunk_tiles;
+          }
+        }
+        sc[0] = b, sc[1] = h, sc[2] = t, sc[3] = (int)blockIdx.x;
+        *srem = rem;
+      }
     }
   } else {
     const long long g0 = range_begin(T, blockIdx.x, a.num_ctas);
@@ -455,7 +478,7 @@ __device__ __forceinline__ bool schedule_prologue(const AttnArgs& a, uint8_t* sm
     }
   }
   __syncthreads();
-  start.cta = a.chunked == 1 ? sc[3] : (int)blockIdx.x;
+  start.cta = (kWalk && a.chunked == 1) ? sc[3] : (int)blockIdx.x;
   start.first = 1;
   start.b = sc[0];
   start.h = sc[1];
@@ -477,7 +500,7 @@ __device__ __forceinline__ bool schedule_prologue(const AttnArgs& a, uint8_t* sm
 // for their ring slots and issue their boxes side by side, one tile per step.
 // Page ids are read four tiles ahead into registers, and the slot and the row
 // inside the page are tracked incrementally (no division per tile).
-template <int D>
+template <int D, bool kWalk>
 __device__ __forceinline__ void producer_role(const AttnArgs& a, uint8_t* smem,
                                               const CUtensorMap* tm_q, const CUtensorMap* tm_kc,
                                               const CUtensorMap* tm_vc, const CUtensorMap* tm_kb,
@@ -504,7 +527,7 @@ __device__ __forceinline__ void producer_role(const AttnArgs& a, uint8_t* smem,
   SegCursor cur = start;
   Segment sg;
   int si = 0;
-  while (ok && cursor_next(a, tab, cur, sg)) {
+  while (ok && cursor_next<kWalk>(a, tab, cur, sg)) {
     const int b = sg.b, h = sg.h;
     const SeqInfo sq = tab.get(a, b);
     const int row0 = sq.row0;
@@ -625,7 +648,7 @@ struct TileStep {
 // Q bookkeeping covers every segment, own tiles or not: at a segment start the
 // warp waits for that unit's Q tile, and after its last QK of the segment it
 // commits one arrival on q_empty (two arrivals, one per warp, release Q).
-template <int D>
+template <int D, bool kWalk>
 __device__ __forceinline__ void mma_role(const AttnArgs& a, uint8_t* smem, uint32_t tmem,
                                          volatile int* abort_flag, int w, const SeqTable& tab,
                                          const SegCursor& start) {
@@ -730,7 +753,7 @@ __device__ __forceinline__ void mma_role(const AttnArgs& a, uint8_t* smem, uint3
   int it0 = 0;  // CTA tile index of the segment's first tile
   int mb = 0;   // own tiles of this warp in earlier segments
   bool ok = true;
-  while (ok && cursor_next(a, tab, cur, sg)) {
+  while (ok && cursor_next<kWalk>(a, tab, cur, sg)) {
     const SeqInfo sq = tab.get(a, sg.b);
     TileStep j;
     j.cur = cur;
@@ -779,7 +802,7 @@ __device__ __forceinline__ void mma_role(const AttnArgs& a, uint8_t* smem, uint3
   __syncwarp();
 }
 
-template <int D>
+template <int D, bool kWalk>
 __device__ __forceinline__ void softmax_role(const AttnArgs& a, uint8_t* smem, uint32_t tmem,
                                              volatile int* abort_flag, const SeqTable& tab,
                                              const SegCursor& start) {
@@ -810,7 +833,7 @@ __device__ __forceinline__ void softmax_role(const AttnArgs& a, uint8_t* smem, u
   Segment sg;
   int it = 0, si = 0;
   bool ok = true;
-  while (ok && cursor_next(a, tab, cur, sg)) {
+  while (ok && cursor_next<kWalk>(a, tab, cur, sg)) {
     const int b = sg.b, h = sg.h;
     const SeqInfo sq = tab.get(a, b);
     const int Kb = sq.Kb, row0 = sq.row0;
@@ -1018,14 +1041,14 @@ __device__ __forceinline__ void softmax_role(const AttnArgs& a, uint8_t* smem, u
 // masks keys at or past L_b and zeroes their V rows), so the copy runs next to
 // the pipeline with no ordering against it. A row whose page index or page id
 // is out of range is skipped and flagged. No waits.
-template <int D>
+template <int D, bool kWalk>
 __device__ __forceinline__ void block_writer_role(const AttnArgs& a, const SeqTable& tab,
                                                   SegCursor c) {
   constexpr int kChunks = D / 8;  // 16-byte chunks per head row
   constexpr int U = 8;            // chunk pairs in flight per lane
   const int lane = threadIdx.x & 31;
   Segment sg;
-  while (cursor_next(a, tab, c, sg)) {
+  while (cursor_next<kWalk>(a, tab, c, sg)) {
     if (sg.t1 != sg.nt) continue;  // another CTA owns this unit's block tile
     const SeqInfo si = tab.get(a, sg.b);
     const int items = si.Kb * kChunks;
@@ -1071,7 +1094,7 @@ __device__ __forceinline__ void block_writer_role(const AttnArgs& a, const SeqTa
   }
 }
 
-template <int D>
+template <int D, bool kWalk>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     block_attn_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_kc,
@@ -1093,7 +1116,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   // A CTA whose range is empty has nothing to set up.
   SeqTable tab;
   SegCursor start;
-  if (!schedule_prologue<D>(a, smem, tab, start)) return;
+  if (!schedule_prologue<D, kWalk>(a, smem, tab, start)) return;
 
   if (threadIdx.x == 0) {
     const uint32_t bars = smem_u32(smem) + Lay::kBarOff;
@@ -1147,9 +1170,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   if (warp == kProducerWarp) {
     if ((threadIdx.x & 31) < 2)
-      producer_role<D>(a, smem, &tm_q, &tm_kc, &tm_vc, &tm_kb, &tm_vb, abort_flag, tab, start);
+      producer_role<D, kWalk>(a, smem, &tm_q, &tm_kc, &tm_vc, &tm_kb, &tm_vb, abort_flag, tab, start);
   } else if (warp < kSoftmaxWarp0) {
-    mma_role<D>(a, smem, tmem, abort_flag, warp - kMmaWarp0, tab, start);
+    mma_role<D, kWalk>(a, smem, tmem, abort_flag, warp - kMmaWarp0, tab, start);
   } else if (warp == kWriterWarp) {
     if (a.write_block) {
       // Start the copies once this CTA's first K tile has landed, off the
@@ -1158,10 +1181,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       // bounded like every other; it gives up only if the pipeline stalled.
       mbar_wait(smem_u32(smem) + Lay::kBarOff + 8u * Lay::kBarKFull, 0, abort_flag,
                 a.timeout_ns);
-      block_writer_role<D>(a, tab, start);
+      block_writer_role<D, kWalk>(a, tab, start);
     }
   } else {
-    softmax_role<D>(a, smem, tmem, abort_flag, tab, start);
+    softmax_role<D, kWalk>(a, smem, tmem, abort_flag, tab, start);
   }
 
   tc_fence_before();

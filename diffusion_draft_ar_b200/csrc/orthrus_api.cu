@@ -271,8 +271,11 @@ orthrus_status_t launch_attn(const orthrus_attn_params* p, const AttnPlan& pl, i
   using Lay = AttnLayout<D>;
   static std::atomic<int> smem_set[kMaxDevices];
   if (!smem_set[dev].load()) {
-    cudaError_t e = cudaFuncSetAttribute(block_attn_kernel<D>,
+    cudaError_t e = cudaFuncSetAttribute(block_attn_kernel<D, false>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kAlloc);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(block_attn_kernel<D, true>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kAlloc);
     if (e != cudaSuccess)
       return fail(ORTHRUS_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
     smem_set[dev].store(1);
@@ -341,7 +344,15 @@ orthrus_status_t launch_attn(const orthrus_attn_params* p, const AttnPlan& pl, i
   a.kc_rows = static_cast<uint4*>(const_cast<void*>(p->k_cache));
   a.vc_rows = static_cast<uint4*>(const_cast<void*>(p->v_cache));
 
-  block_attn_kernel<D><<<pl.grid, kAttnThreads, Lay::kAlloc, stream>>>(tq, tkc, tvc, tkb, tvb, a);
+  // Fixed-chunk CTAs that walk several slots run the walking variant; every
+  // other schedule (one slot per CTA included) runs the variant without it.
+  const bool walk = pl.chunked == 1 && pl.grid < pl.parts;
+  if (walk)
+    block_attn_kernel<D, true><<<pl.grid, kAttnThreads, Lay::kAlloc, stream>>>(tq, tkc, tvc, tkb,
+                                                                              tvb, a);
+  else
+    block_attn_kernel<D, false><<<pl.grid, kAttnThreads, Lay::kAlloc, stream>>>(tq, tkc, tvc, tkb,
+                                                                               tvb, a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return fail(ORTHRUS_ERR_CUDA, "block_attn launch: %s", cudaGetErrorString(e));
   if (!pl.combine) return ok();
