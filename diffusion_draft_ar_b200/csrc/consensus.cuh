@@ -171,32 +171,36 @@ __device__ __forceinline__ Philox4 philox4x32_10(uint32_t c0, uint32_t c1, uint3
   return Philox4{c0, c1, c2, c3};
 }
 
-// -ln(-ln u) for u = (k + 1/2) / 2^24, k = word >> 8. e = -ln u must be
-// accurate in relative terms, since g = -ln e. For u < 15/16, |log2 u| >= 0.09
-// and the hardware base-2 logarithm (absolute error ~2^-22) gives e to ~3e-6.
-// For u >= 15/16 (where the largest noise values, the likely winners, come
-// from) e is the series of -ln(1 - v) = v + v^2/2 + v^3/3 + ... in v = 1 - u,
-// which is exact in fp32; seven terms leave a relative error below v^7/8 <=
-// 2^-31. The outer logarithm needs only absolute accuracy (~2e-7 in g).
-// Both forms are evaluated and one is selected: in nearly every warp some
-// lane needs the series, so a branch would run both anyway, converting k
-// twice (one conversion here; v = 2^24 - k - 1/2 is exact for the series
-// lanes).
-__device__ __forceinline__ float gumbel_noise(uint32_t word) {
+// The kernel ranks base-2 scores. With e = -ln u, the Gumbel-max score
+// s = x / T - ln e divided by ln 2 is x log2(e) / T - log2(ln 2) - log2(a)
+// with a = e / ln 2 = -log2 u; the constant is the same for every entry, so
+// r = x * x_scale - log2(a), x_scale = log2(e) / T, has the same argmax.
+// noise_log2 returns -log2(a) for u = (k + 1/2) / 2^24, k = word >> 8. a must
+// be accurate in relative terms. For u < 15/16, |log2 u| >= 0.09 and the
+// hardware base-2 logarithm (absolute error ~2^-22) gives a to ~3e-6. For
+// u >= 15/16 (where the largest noise values, the likely winners, come from)
+// a is the series of -log2(1 - v) = (v + v^2/2 + v^3/3 + ...) / ln 2 in
+// v = 1 - u, which is exact in fp32; seven terms leave a relative error below
+// v^7/8 <= 2^-31. The outer logarithm needs only absolute accuracy. Both
+// forms are evaluated and one is selected: in nearly every warp some lane
+// needs the series, so a branch would run both anyway. Emulated in fp32
+// against fp64 over every series k and 2M sampled log-branch k, the result
+// is within 2e-7 and 8e-7 (base-2 units) of -log2(-log2 u).
+__device__ __forceinline__ float noise_log2(uint32_t word) {
   const uint32_t k = word >> 8;
   const float kf = static_cast<float>(k);
-  const float v = ((16777216.f - kf) - 0.5f) * 5.9604644775390625e-8f;  // 2^-24
-  float q = fmaf(v, 1.f / 7.f, 1.f / 6.f);
-  q = fmaf(v, q, 0.2f);
-  q = fmaf(v, q, 0.25f);
-  q = fmaf(v, q, 1.f / 3.f);
-  q = fmaf(v, q, 0.5f);
-  q = fmaf(v, q, 1.f);
-  const float e_series = v * q;
-  const float u = (kf + 0.5f) * 5.9604644775390625e-8f;
-  const float e_log = -0.6931471805599453f * __log2f(u);
-  const float e = (k >= (15u << 20)) ? e_series : e_log;
-  return -0.6931471805599453f * __log2f(e);
+  const float v = ((16777216.f - kf) - 0.5f) * 5.9604644775390625e-8f;  // exact: v = m / 2^25
+  float q = fmaf(v, 2.060992867e-01f, 2.404491752e-01f);  // 1 / (j ln 2), j = 7, 6
+  q = fmaf(v, q, 2.885390222e-01f);                       // j = 5
+  q = fmaf(v, q, 3.606737554e-01f);                       // j = 4
+  q = fmaf(v, q, 4.808983505e-01f);                       // j = 3
+  q = fmaf(v, q, 7.213475108e-01f);                       // j = 2
+  q = fmaf(v, q, 1.442695022e+00f);                       // j = 1
+  const float a_series = v * q;
+  const float u = fmaf(kf, 5.9604644775390625e-8f, 2.98023223876953125e-8f);  // (k + 1/2) 2^-24
+  const float a_log = -__log2f(u);
+  const float a = (k >= (15u << 20)) ? a_series : a_log;
+  return -__log2f(a);
 }
 
 // One CTA per (row, 16,384-entry chunk): every thread takes groups of four
@@ -211,7 +215,7 @@ __device__ __forceinline__ float gumbel_noise(uint32_t word) {
 __global__ void __launch_bounds__(kConsThreads)
     consensus_sample_kernel(const float* __restrict__ logits, long long ld, int V,
                             const int* __restrict__ cu_block, int B, int max_block, int n_chunks,
-                            unsigned long long* __restrict__ part, float inv_t, uint32_t seed_lo,
+                            unsigned long long* __restrict__ part, float x_scale, uint32_t seed_lo,
                             uint32_t seed_hi, uint32_t off_lo, uint32_t off_hi) {
   pdl_launch_dependents();  // the finalize pass may start its launch now
   const int r = blockIdx.y;
@@ -240,10 +244,10 @@ __global__ void __launch_bounds__(kConsThreads)
                                     off_hi, seed_lo, seed_hi);
     if (bidx < 0) bidx = v;  // lowest index this thread sees: the tie default
     float sc[4];
-    sc[0] = fmaf(x[0], inv_t, gumbel_noise(w.x));
-    sc[1] = fmaf(x[1], inv_t, gumbel_noise(w.y));
-    sc[2] = fmaf(x[2], inv_t, gumbel_noise(w.z));
-    sc[3] = fmaf(x[3], inv_t, gumbel_noise(w.w));
+    sc[0] = fmaf(x[0], x_scale, noise_log2(w.x));
+    sc[1] = fmaf(x[1], x_scale, noise_log2(w.y));
+    sc[2] = fmaf(x[2], x_scale, noise_log2(w.z));
+    sc[3] = fmaf(x[3], x_scale, noise_log2(w.w));
     const float m = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3]));
     if (m > best) {
       best = m;

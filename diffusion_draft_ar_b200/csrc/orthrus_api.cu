@@ -539,8 +539,9 @@ orthrus_status_t orthrus_consensus_sampled(const float* verify_logits, int64_t l
   if (!(temperature > 0.f) || !std::isfinite(temperature))
     return fail(ORTHRUS_ERR_INVALID_ARG, "temperature = %g (must be finite and > 0)",
                 static_cast<double>(temperature));
-  const float inv_t = 1.f / temperature;
-  if (!std::isfinite(inv_t))
+  // base-2 scores: logits scaled by log2(e) / T (see noise_log2)
+  const float x_scale = static_cast<float>(1.4426950408889634 / static_cast<double>(temperature));
+  if (!std::isfinite(x_scale))
     return fail(ORTHRUS_ERR_UNSUPPORTED, "temperature = %g is too small for fp32 scores",
                 static_cast<double>(temperature));
   if (B < 0) return fail(ORTHRUS_ERR_INVALID_ARG, "B = %d < 0", B);
@@ -561,7 +562,7 @@ orthrus_status_t orthrus_consensus_sampled(const float* verify_logits, int64_t l
   auto* part = static_cast<unsigned long long*>(workspace);
   dim3 grid(n_chunks, static_cast<unsigned>(R_max));
   consensus_sample_kernel<<<grid, kConsThreads, 0, st>>>(
-      verify_logits, ld, V, cu_block, B, max_block, n_chunks, part, inv_t,
+      verify_logits, ld, V, cu_block, B, max_block, n_chunks, part, x_scale,
       static_cast<uint32_t>(seed), static_cast<uint32_t>(seed >> 32),
       static_cast<uint32_t>(offset), static_cast<uint32_t>(offset >> 32));
   cudaError_t e = cudaGetLastError();
