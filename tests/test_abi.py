@@ -124,14 +124,27 @@ def test_block_attn_empty_batch_is_a_no_op(O):
 
 
 def test_block_attn_workspace_size_chunked_mode(O):
-    # fixed 2048-token chunks: one partial per CTA, grid = chunks * Hkv * B
+    # fixed 2048-token chunks: one partial slot per (unit, chunk), whatever the
+    # number of CTAs that walk the slots (max_ctas only caps that grid)
     p = _params(O, B=1, Hq=32, Hkv=8, max_block=32, total_rows=32, max_pages_per_seq=2049,
                 num_pages=2049, kv_split_tokens=2048)
     n = O.block_attn_workspace_size(p)
     chunks = -(-2049 * 64 // 2048)
     parts = chunks * 8
     assert n == parts * 128 * 128 * 4 + (-(-parts * 128 * 4 // 256)) * 256
+    for cap in (1, 7, 130, 10 ** 6):
+        p.max_ctas = cap
+        assert O.block_attn_workspace_size(p) == n
     assert O.block_attn_workspace_size(_params(O, D=96, kv_split_tokens=64)) == 0
+
+
+def test_block_attn_balanced_workspace_holds_two_partials_per_cta(O):
+    # balanced ranges over max_ctas CTAs: a CTA's first and last segments may
+    # each be a partial
+    for cap in (1, 7, 148):
+        n = O.block_attn_workspace_size(_params(O, max_ctas=cap))
+        parts = 2 * cap
+        assert n == parts * 128 * 128 * 4 + (-(-parts * 128 * 4 // 256)) * 256
 
 
 def test_block_attn_kernel_count(O):
