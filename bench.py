@@ -31,6 +31,7 @@ import ctypes
 import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -157,15 +158,25 @@ def measure_lm_head(O, w: W.Workload, m: W.BatchMeta, dev, stream, calls: int = 
                                            "consensus finalize; logits never written"}
 
 
+def kernel_code_hash(path) -> str:
+    """First 16 hex digits of the sha256 of a CUDA source with its comments,
+    indentation and blank lines removed: edits to comments keep the hash, any
+    change to the code changes it."""
+    text = open(path, encoding="utf-8").read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    lines = (re.sub(r"//.*", "", ln).strip() for ln in text.splitlines())
+    code = "\n".join(ln for ln in lines if ln)
+    return hashlib.sha256(code.encode()).hexdigest()[:16]
+
+
 def traffic_per_launch():
     """DRAM bytes per attention launch from the committed ncu figures
     (profiles/block_attn_qwen3_8b.json), or None when they are missing or were
-    taken on a different kernel source."""
+    taken on different kernel code."""
     try:
         with open(TRAFFIC_FILE) as f:
             d = json.load(f)
-        src_hash = hashlib.sha256(open(ATTN_SRC, "rb").read()).hexdigest()[:16]
-        if d.get("kernel_source_sha256_16") == src_hash:
+        if d.get("kernel_code_sha256_16") == kernel_code_hash(ATTN_SRC):
             return int(d["dram_bytes_per_launch_full_size"])
     except Exception:
         pass

@@ -11,10 +11,14 @@
 // Work unit = (sequence b, KV head h). Its G*K_b query rows (token-major:
 // row r = i*G + g) form one M = 128 MMA tile that stays in shared memory; the
 // unit's keys are cut into 64-key tiles: ceil(L_b/64) prefix tiles, then one
-// block tile. A CTA (one per SM) walks a contiguous range of the global
-// (unit, tile) sequence, so every CTA gets the same number of tiles whatever
-// the prefix lengths; a unit cut by a range boundary is finished by the combine
-// kernel from per-CTA partials (max, sum, normalised accumulator).
+// block tile. The host picks one of four schedules (see plan_attn): one CTA
+// per whole unit; proportional chunks (few long units, each cut into
+// near-equal chunks in proportion to its tiles); balanced ranges (a CTA per SM
+// walks a contiguous range of the global (unit, tile) sequence, so every CTA
+// gets the same number of tiles whatever the prefix lengths); or fixed chunks
+// of a given number of tokens, walked by at most one CTA per SM. A unit that
+// is cut is finished by the combine kernel from the partials (max, sum,
+// normalised accumulator) of its pieces.
 //
 // Roles (384 threads):
 //   warp 0      TMA producer, two lanes: lane 0 issues the Q tile per unit

@@ -54,23 +54,25 @@ def test_consensus_and_append_bytes(q8):
     assert bench.append_bytes(w, 1) == 2 * 2 * w.Hkv * w.D * 2 == 8192
 
 
-def test_traffic_file_follows_the_kernel_hash(monkeypatch):
+def test_traffic_file_follows_the_kernel_code(monkeypatch):
     """The bench reports DRAM traffic only while the committed ncu figures were
-    taken on the current kernel source."""
-    import hashlib
+    taken on the current kernel code: a comment edit keeps them, a code edit
+    drops them."""
     import json
-    src = b"// kernel source\n"
-    h = hashlib.sha256(src).hexdigest()[:16]
+    src = "// kernel source\n__global__ void k(int* p) {\n  p[0] = 1;  // store\n}\n"
     with tempfile.TemporaryDirectory() as d:
         k = os.path.join(d, "k.cuh")
-        open(k, "wb").write(src)
+        open(k, "w").write(src)
+        h = bench.kernel_code_hash(k)
         s = os.path.join(d, "s.json")
-        json.dump({"kernel_source_sha256_16": h, "dram_bytes_per_launch_full_size": 1234},
+        json.dump({"kernel_code_sha256_16": h, "dram_bytes_per_launch_full_size": 1234},
                   open(s, "w"))
         monkeypatch.setattr(bench, "ATTN_SRC", k)
         monkeypatch.setattr(bench, "TRAFFIC_FILE", s)
         assert bench.traffic_per_launch() == 1234
-        open(k, "wb").write(src + b"// changed\n")
+        open(k, "w").write("/* header */\n" + src.replace("// store", "// the store") + "\n\n")
+        assert bench.traffic_per_launch() == 1234
+        open(k, "w").write(src.replace("p[0] = 1;", "p[0] = 2;"))
         assert bench.traffic_per_launch() is None
 
 
