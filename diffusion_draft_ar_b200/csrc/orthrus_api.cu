@@ -404,6 +404,26 @@ int32_t orthrus_block_attn_kernel_count(const orthrus_attn_params* p) {
   return pl.combine ? 2 : 1;
 }
 
+orthrus_status_t orthrus_block_attn_plan(const orthrus_attn_params* p, int32_t sm_count,
+                                         orthrus_attn_plan* plan) {
+  if (!plan) return fail(ORTHRUS_ERR_INVALID_ARG, "plan is NULL");
+  int sms = sm_count;
+  if (sms <= 0 && device_sm_count(&sms) < 0) return fail(ORTHRUS_ERR_CUDA, "no current CUDA device");
+  AttnPlan pl;
+  const orthrus_status_t s = plan_attn(p, sms, &pl);
+  if (s != ORTHRUS_OK) return s;
+  plan->schedule = pl.chunked == 2   ? ORTHRUS_SCHEDULE_PROPORTIONAL
+                   : pl.chunked == 1 ? ORTHRUS_SCHEDULE_FIXED_CHUNKS
+                                     : ORTHRUS_SCHEDULE_BALANCED;
+  plan->grid = pl.grid;
+  plan->partial_slots = pl.parts;
+  plan->kernels = pl.combine ? 2 : 1;
+  plan->walks_chunks = (pl.chunked == 1 && pl.grid < pl.parts) ? 1 : 0;  // as launch_attn
+  plan->chunk_tiles = pl.chunked == 1 ? pl.chunk_tiles : 0;
+  plan->workspace_bytes = pl.ws_bytes;
+  return ok();
+}
+
 static orthrus_status_t block_attn_entry(const orthrus_attn_params* p, void* stream, bool write_block) {
   AttnPlan pl;
   orthrus_status_t s = plan_attn(p, 1, &pl);  // geometry checks first, no CUDA call

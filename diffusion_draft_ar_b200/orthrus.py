@@ -46,8 +46,20 @@ class AttnParams(ctypes.Structure):
     ]
 
 
+class AttnPlan(ctypes.Structure):
+    """Mirror of ``orthrus_attn_plan``."""
+    _fields_ = [
+        ("schedule", _i32), ("grid", _i32), ("partial_slots", _i32), ("kernels", _i32),
+        ("walks_chunks", _i32), ("chunk_tiles", _i32), ("workspace_bytes", _sz),
+    ]
+
+
+SCHEDULES = {0: "balanced", 1: "fixed_chunks", 2: "proportional"}
+
 lib.orthrus_block_attn_workspace_size.restype = _sz
 lib.orthrus_block_attn_workspace_size.argtypes = [ctypes.POINTER(AttnParams)]
+lib.orthrus_block_attn_plan.restype = _i32
+lib.orthrus_block_attn_plan.argtypes = [ctypes.POINTER(AttnParams), _i32, ctypes.POINTER(AttnPlan)]
 lib.orthrus_block_attn_kernel_count.restype = _i32
 lib.orthrus_block_attn_kernel_count.argtypes = [ctypes.POINTER(AttnParams)]
 lib.orthrus_block_attn.restype = _i32
@@ -161,6 +173,15 @@ def block_attn_workspace_size(params: AttnParams) -> int:
 def block_attn_kernel_count(params: AttnParams) -> int:
     """Kernels one ``orthrus_block_attn`` call with these parameters launches."""
     return int(lib.orthrus_block_attn_kernel_count(ctypes.byref(params)))
+
+
+def block_attn_plan(params: AttnParams, sm_count: int = 0) -> AttnPlan:
+    """``orthrus_block_attn_plan``: the schedule a call with these parameters
+    uses on ``sm_count`` SMs (0: the current device's)."""
+    plan = AttnPlan()
+    _check(lib.orthrus_block_attn_plan(ctypes.byref(params), int(sm_count), ctypes.byref(plan)),
+           "orthrus_block_attn_plan")
+    return plan
 
 
 def block_attn(view, q_block, k_cache, v_cache, k_block, v_block, prefix_lens, cu_block,

@@ -160,6 +160,32 @@ ORTHRUS_API size_t orthrus_block_attn_workspace_size(const orthrus_attn_params* 
  * that merges the partials). 0 when the parameters are invalid. */
 ORTHRUS_API int32_t orthrus_block_attn_kernel_count(const orthrus_attn_params* p);
 
+/* The schedule orthrus_block_attn picks for *p, decided on the host from the
+ * parameters alone: the kernels then cut proportional chunks and balanced
+ * ranges from the actual prefix lengths on the device.
+ *   sm_count  SMs to plan for; <= 0: the current device's (a CUDA query).
+ * Returns OK and fills *plan, or INVALID_ARG / UNSUPPORTED as orthrus_block_attn
+ * would for these parameters (plan NULL: INVALID_ARG), or CUDA when sm_count
+ * <= 0 and there is no current device. No allocation, no launch. */
+typedef enum {
+  ORTHRUS_SCHEDULE_BALANCED = 0,     /* one contiguous range of the (unit, tile) list per CTA */
+  ORTHRUS_SCHEDULE_FIXED_CHUNKS = 1, /* kv_split_tokens chunks, or one chunk per whole unit */
+  ORTHRUS_SCHEDULE_PROPORTIONAL = 2  /* few units, each cut in proportion to its tiles */
+} orthrus_schedule_t;
+
+typedef struct {
+  int32_t schedule;        /* orthrus_schedule_t */
+  int32_t grid;            /* attention CTAs */
+  int32_t partial_slots;   /* (max, sum, accumulator) partial slots the workspace holds */
+  int32_t kernels;         /* launches per call: 1 (no unit cut) or 2 (attention, combine) */
+  int32_t walks_chunks;    /* 1: fixed-chunk CTAs take several chunk slots each */
+  int32_t chunk_tiles;     /* fixed chunks: 64-key prefix tiles per chunk; else 0 */
+  size_t workspace_bytes;  /* as orthrus_block_attn_workspace_size for this SM count */
+} orthrus_attn_plan;
+
+ORTHRUS_API orthrus_status_t orthrus_block_attn_plan(const orthrus_attn_params* p,
+                                                     int32_t sm_count, orthrus_attn_plan* plan);
+
 /* Launch the block attention described by *p on `stream`.
  * q_block, k_block, v_block and out hold total_rows rows; a sequence whose
  * cu_block range is decreasing, longer than max_block or past total_rows is

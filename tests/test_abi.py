@@ -257,3 +257,80 @@ def test_sampled_consensus_rejects_bad_temperatures_on_the_host(O, T):
                                          None, None, ctypes.c_void_p(16), 1 << 20, None)
     assert st in (O.ERR_INVALID_ARG, O.ERR_UNSUPPORTED)
     assert b"temperature" in O.lib.orthrus_last_error()
+
+
+def test_plan_struct_layout_matches_header(O):
+    fields = [f[0] for f in O.AttnPlan._fields_]
+    prog = ["#include <stdio.h>", "#include <stddef.h>", '#include "orthrus.h"', "int main(void){",
+            'printf("%zu\\n", sizeof(orthrus_attn_plan));']
+    prog += [f'printf("%zu\\n", offsetof(orthrus_attn_plan, {f}));' for f in fields]
+    prog.append("return 0;}")
+    with tempfile.TemporaryDirectory() as d:
+        c = os.path.join(d, "plan.c")
+        exe = os.path.join(d, "plan")
+        open(c, "w").write("\n".join(prog))
+        subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), "-o", exe, c], check=True)
+        vals = [int(x) for x in subprocess.run([exe], capture_output=True, text=True,
+                                                check=True).stdout.split()]
+    assert vals[0] == ctypes.sizeof(O.AttnPlan)
+    for f, off in zip(fields, vals[1:]):
+        assert getattr(O.AttnPlan, f).offset == off, f
+
+
+def _shape(O, B, max_pages, max_block=32, **kw):
+    """Qwen3-8B-like heads (32 / 8, D = 128) with B sequences of up to
+    max_pages 64-token pages."""
+    return _params(O, B=B, Hq=32, Hkv=8, D=128, max_block=max_block, total_rows=B * max_block,
+                   max_pages_per_seq=max_pages, num_pages=B * max_pages, **kw)
+
+
+@pytest.mark.parametrize("name,B,pages,kw,want", [
+    # 16 x 8192-token prefixes: 128 units on 148 SMs, one CTA per whole unit
+    ("qwen3_8b", 16, 129, {}, dict(schedule=1, grid=128, partial_slots=128, kernels=1,
+                                   walks_chunks=0, chunk_tiles=129)),
+    # one 131,072-token prefix: 8 units cut in proportion over all SMs
+    ("longctx", 1, 2049, {}, dict(schedule=2, grid=148, partial_slots=148, kernels=2,
+                                   walks_chunks=0, chunk_tiles=0)),
+    # the same in 2048-token chunks: 520 slots spread 4 per CTA over 130 walkers
+    ("longctx_2048", 1, 2049, dict(kv_split_tokens=2048),
+     dict(schedule=1, grid=130, partial_slots=520, kernels=2, walks_chunks=1, chunk_tiles=32)),
+    # ... or over an explicit cap
+    ("longctx_2048_cap", 1, 2049, dict(kv_split_tokens=2048, max_ctas=7),
+     dict(schedule=1, grid=7, partial_slots=520, kernels=2, walks_chunks=1, chunk_tiles=32)),
+    # 64 sequences: 512 units > 148 SMs, balanced ranges (two partial slots per CTA)
+    ("ragged", 64, 517, {}, dict(schedule=0, grid=148, partial_slots=296, kernels=2,
+                                  walks_chunks=0, chunk_tiles=0)),
+    # an explicit CTA count is a balanced split
+    ("capped", 16, 129, dict(max_ctas=37), dict(schedule=0, grid=37, partial_slots=74, kernels=2,
+                                                 walks_chunks=0, chunk_tiles=0)),
+    # few units, none long enough to cut (under 8 tiles): one CTA each, no combine
+    ("short", 1, 1, dict(max_block=8), dict(schedule=2, grid=8, partial_slots=8, kernels=1,
+                                            walks_chunks=0, chunk_tiles=0)),
+])
+def test_schedule_plans(O, name, B, pages, kw, want):
+    p = _shape(O, B, pages, **kw)
+    plan = O.block_attn_plan(p, 148)
+    got = {k: getattr(plan, k) for k in want}
+    assert got == want, name
+    if p.kv_split_tokens > 0 or p.max_ctas > 0:  # no device query needed
+        assert plan.workspace_bytes == O.block_attn_workspace_size(p)
+        assert plan.kernels == O.block_attn_kernel_count(p)
+    slots = plan.partial_slots
+    assert plan.workspace_bytes == slots * 128 * 128 * 4 + -(-slots * 128 * 4 // 256) * 256
+
+
+def test_plan_follows_the_sm_count(O):
+    p = _shape(O, 16, 129)
+    # 128 units: one CTA each from 128 SMs up to 171 (floor(3 * 171 / 4) = 128)
+    assert O.block_attn_plan(p, 128).schedule == 1
+    assert O.block_attn_plan(p, 171).schedule == 1
+    assert O.block_attn_plan(p, 172).schedule == 2   # fewer units than 3/4 of the SMs
+    assert O.block_attn_plan(p, 127).schedule == 0   # more units than SMs
+    assert O.block_attn_plan(p, 127).grid == 127
+
+
+def test_plan_refuses_what_the_call_refuses(O):
+    with pytest.raises(O.OrthrusError) as e:
+        O.block_attn_plan(_params(O, D=96), 148)
+    assert e.value.status == O.ERR_UNSUPPORTED
+    assert O.lib.orthrus_block_attn_plan(ctypes.byref(_params(O)), 148, None) == O.ERR_INVALID_ARG
