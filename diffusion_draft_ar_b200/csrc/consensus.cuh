@@ -184,8 +184,8 @@ __device__ __forceinline__ Philox4 philox4x32_10(uint32_t c0, uint32_t c1, uint3
 // v^7/8 <= 2^-31. The outer logarithm needs only absolute accuracy. Both
 // forms are evaluated and one is selected: in nearly every warp some lane
 // needs the series, so a branch would run both anyway. Emulated in fp32
-// against fp64 over every series k and 2M sampled log-branch k, the result
-// is within 2e-7 and 8e-7 (base-2 units) of -log2(-log2 u).
+// against fp64 over every series k and a million sampled log-branch k, the
+// result is within 2e-7 and 8e-7 (base-2 units) of -log2(-log2 u).
 __device__ __forceinline__ float noise_log2(uint32_t word) {
   const uint32_t k = word >> 8;
   const float kf = static_cast<float>(k);
